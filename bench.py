@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Sparse-prefill benchmark on B200: tokens/s of one block-sparse attention
+prefill (pool -> select -> attend) at 128k tokens, the RBS dual-branch
+workload (32 query / 8 kv heads, d = 128, B = 128, bf16, cumulative score
+mass 0.9 united with the radius rescue branch).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sbsa|reference]
+
+One process per GPU (torchrun for N > 1).  Every rank runs its own
+independent sequence (weak scaling, no collective on the data path); the
+reported time is the maximum over ranks.  Rank 0 prints one JSON line.
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse prefill tokens/s and attended TFLOP/s at 128k; % of bf16 TC / HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch, from the
+# ncu capture summarised in profiles/ (None until captured for this kernel).
+NCU_ATTEND_TRAFFIC = {}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="sbsa", choices=["sbsa", "reference"])
+    ap.add_argument("--workload", default="rbs128k")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-blocks", type=int, default=6,
+                    help="query blocks (all heads) in the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = list(csv.reader(io.StringIO(self.tmp.read())))
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------- CPU oracle leg
+def oracle_sample(w, data_cpu, blocks):
+    """Oracle work for the full key pooling plus selection and attention of
+    the given query blocks (all heads).  Returns (t_pool, t_rows) seconds."""
+    import numpy as np
+    import oracle as O
+    t0 = time.perf_counter()
+    ks = data_cpu["k_idx"] if w.index_dim else data_cpu["k"]
+    c, r = O.pool_keys(ks, w.block_size, with_radius=w.rescue_tau is not None)
+    if r is None:
+        r = np.zeros(c.shape[:2])
+    t_pool = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    nb, b = w.n_blocks, w.block_size
+    grp = w.group if w.group_shared else 1
+    qbar = np.zeros((w.n_sel_heads, nb, w.score_dim))
+    qsrc = data_cpu["q_rows_idx"] if w.index_dim else data_cpu["q_rows"]
+    for bi, i in enumerate(blocks):
+        qbar[:, i] = O.pool_queries(qsrc[:, bi * b:(bi + 1) * b], b, group=grp)[:, 0]
+    kv_of = (lambda hs: hs) if w.group_shared else (lambda hs: hs // w.group)
+    rows = [(hs, i) for hs in range(w.n_sel_heads) for i in blocks]
+    idx, cnt, _ = O.select(qbar, c, r, block_count=nb, mode=w.select_mode, top_k_=w.top_k,
+                           mass=w.mass_threshold, margin=w.gate_margin, tau=w.rescue_tau,
+                           scale=1.0 / math.sqrt(w.score_dim), kv_of_sel=kv_of,
+                           max_blocks=w.max_blocks, rows=rows)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    for bi, i in enumerate(blocks):
+        for h in range(w.n_q_heads):
+            hs = h // w.group if w.group_shared else h
+            ids = [int(x) for x in idx[hs, i, :cnt[hs, i]]]
+            O.attend_block(data_cpu["q_rows"][h, bi * b:(bi + 1) * b], data_cpu["k"][h // w.group],
+                           data_cpu["v"][h // w.group], ids, i, b, scale)
+    t_rows = time.perf_counter() - t1
+    return t_pool, t_rows
+
+
+def cpu_copy_for_oracle(w, data, blocks):
+    import torch
+    b = w.block_size
+    out = {"k": data["k"].cpu(), "v": data["v"].cpu(),
+           "k_idx": data["k_idx"].cpu() if data["k_idx"] is not None else None}
+    out["q_rows"] = torch.cat([data["q"][:, i * b:(i + 1) * b] for i in blocks], dim=1).cpu()
+    if data["q_idx"] is not None:
+        out["q_rows_idx"] = torch.cat([data["q_idx"][:, i * b:(i + 1) * b] for i in blocks],
+                                      dim=1).cpu()
+    return out
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((d.get("num_threads", 1) for d in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def sample_blocks(w, count, salt=0):
+    import torch
+    g = torch.Generator().manual_seed(w.seed + 101 + salt)
+    picks = set()
+    while len(picks) < min(count, w.n_blocks):
+        picks.add(int(torch.randint(0, w.n_blocks, (1,), generator=g)))
+    return sorted(picks)
+
+
+def cpu_baseline_value(w, data, nblocks):
+    blocks = sample_blocks(w, nblocks)
+    cdata = cpu_copy_for_oracle(w, data, blocks)
+    t_pool, t_rows = oracle_sample(w, cdata, blocks)
+    full = t_pool + t_rows * w.n_blocks / len(blocks)
+    return {
+        "value": w.seq_len / full, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        "sample": (f"numpy float64 oracle: key pooling of all {w.n_blocks} blocks "
+                   f"({t_pool:.1f}s) + selection and attention of {len(blocks)} query blocks x "
+                   f"{w.n_q_heads} heads ({t_rows:.1f}s), extrapolated per query block to the "
+                   f"full {w.seq_len}-token prefill ({full:.0f}s)"),
+    }
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    import torch
+    from block_sparse_attention_sbsa_b200 import workloads as W
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.CONFIGS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    data = W.generate(w, dev)
+    total_t, total_tok = 0.0, 0
+    for s in range(args.warmup + args.steps):
+        blocks = sample_blocks(w, 1, salt=s)
+        cdata = cpu_copy_for_oracle(w, data, blocks)
+        t_pool, t_rows = oracle_sample(w, cdata, blocks)
+        if s >= args.warmup:
+            total_t += t_pool + t_rows * w.n_blocks / len(blocks)
+            total_tok += w.seq_len
+    value = total_tok / total_t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * total_t / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": ("per step: key pooling of all blocks + selection and "
+                                    "attention of 1 query block x all heads, extrapolated per "
+                                    "query block to the full prefill")},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "seq_len": w.seq_len, "head_dim": w.head_dim, "block_size": w.block_size,
+            "select": (f"cumulative mass {w.mass_threshold} + rescue tau {w.rescue_tau}"
+                       if w.select_mode == "cummass" else
+                       f"top-{w.top_k}" + (f" gated x2 margin {w.gate_margin}" if w.gate_margin
+                                           else "") + (" per GQA group" if w.group_shared else "")),
+            "global_batch": 1, "seq": w.seq_len,
+            "l2": "inputs larger than L2 (Q, K, V each exceed 126 MB); no flush between steps"}
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_sbsa_b200 import sbsa
+    from block_sparse_attention_sbsa_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+
+    base = W.CONFIGS[args.workload]
+    w = base.scaled(seed=base.seed + 1000 * rank)   # each rank: its own sequence
+    data = W.generate(w, "cuda")
+    p = sbsa.params_for(w)
+    st = sbsa.Staged(p)
+    q, k, v = data["q"], data["k"], data["v"]
+    qs = data["q_idx"] if w.index_dim else q
+    ks = data["k_idx"] if w.index_dim else k
+    o = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        st.pool(qs, ks)
+        if evs:
+            evs[1].record(stream)
+        st.select()
+        if evs:
+            evs[2].record(stream)
+        st.attend(q, k, v, o)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stat = sbsa.get_status()
+    if stat != sbsa.OK:
+        raise RuntimeError(f"device status after warm-up: {sbsa.status_string(stat)}")
+    pairs = sbsa.attended_pairs(p, st.cnt)
+    attend_flops = 4.0 * w.head_dim * pairs
+    mean_cnt = float(st.cnt.float().mean())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    sel_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    att_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    stat = sbsa.get_status()
+    if stat != sbsa.OK:
+        raise RuntimeError(f"device status after timing: {sbsa.status_string(stat)}")
+
+    # ---- end to end through the C ABI with host buffers ----
+    pin = {name: t.cpu().pin_memory() for name, t in
+           (("q", q), ("k", k), ("v", v), ("q_idx", data["q_idx"]), ("k_idx", data["k_idx"]))
+           if t is not None}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    dev_in = {name: torch.empty_like(t, device="cuda") for name, t in pin.items()}
+    pre = sbsa.Prefill(p, keep_lists=False)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step():
+        for name, t in pin.items():
+            dev_in[name].copy_(t, non_blocking=True)
+        pre(dev_in["q"], dev_in["k"], dev_in["v"], dev_in.get("q_idx"), dev_in.get("k_idx"), out=o)
+        o_host.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    stat = sbsa.get_status()
+    if stat != sbsa.OK:
+        raise RuntimeError(f"device status after e2e: {sbsa.status_string(stat)}")
+
+    # ---- max over ranks ----
+    vals = torch.tensor([elapsed_ms, e2e_ms, att_ms, pool_ms, sel_ms], device="cuda",
+                        dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms, att_ms, pool_ms, sel_ms = [float(x) for x in vals.tolist()]
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    peaks, src = load_peaks()
+    tokens = w.seq_len * world * args.steps
+    value = tokens / (elapsed_ms / 1000.0)
+    ms_per_step = elapsed_ms / args.steps
+    att_tflops = attend_flops / (att_ms / 1000.0) / 1e12
+    peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    # algorithmic bytes of pooling + selection: read Q and K (or the index
+    # tensors) once, write the fp32 tables, read them back, write the lists
+    es = q.element_size()
+    nb, hs, ds = w.n_blocks, w.n_sel_heads, w.score_dim
+    tables = 4 * (hs * nb * ds + w.n_kv_heads * nb * ds + (w.n_kv_heads * nb if w.rescue_tau else 0))
+    lists = hs * nb * (4 * w.max_blocks + 4 + 1)
+    sel_bytes = (qs.numel() + ks.numel()) * es + 2 * tables + lists
+    sel_gbs = sel_bytes / ((pool_ms + sel_ms) / 1000.0) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+        "data": "synthetic (seeded generator, RBS-style clustered keys with outliers)",
+        "config": workload_config(w),
+        "attended_tflops": att_tflops,
+        "roofline": {
+            "bound": "tensor", "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",
+            "frac": att_tflops / peak_tf,
+            "traffic": NCU_ATTEND_TRAFFIC.get(w.name),
+            "kernel": "attend_kernel (tcgen05, bf16, B=128, d=128)",
+            "note": f"peak = bf16_tflops burst, of {src}; achieved = 4*d*unmasked pairs / mean launch time",
+        },
+        "selection_roofline": {
+            "bound": "hbm", "achieved": sel_gbs, "peak": peak_bw, "unit": "GB/s",
+            "frac": sel_gbs / peak_bw, "bytes": sel_bytes,
+            "note": f"pool + select kernels; peak = hbm_gbs copy, of {src}",
+        },
+        "stages_ms": {"pool": pool_ms, "select": sel_ms, "attend": att_ms},
+        "selected_blocks_per_row": mean_cnt,
+        "attended_pairs": pairs,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+        "e2e": {"value": w.seq_len * world * args.e2e_steps / (e2e_ms / 1000.0), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "pinned host -> device copies, sbsa_prefill, device -> host copy of O"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_value(w, data, args.cpu_blocks)
+    print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

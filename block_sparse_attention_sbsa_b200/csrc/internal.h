@@ -1,0 +1,71 @@
+// Internal interfaces between the C-ABI layer and the kernel launchers.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/sbsa.h"
+
+namespace sbsa {
+
+// One pooling job: x [n_heads, N, dim] -> centroids [n_heads/group, NB, dim]
+// (+ radii [n_heads, NB] when rad != nullptr and group == 1).
+struct PoolJob {
+  const void* x;
+  int n_heads;
+  int group;
+  float* cent;
+  float* rad;
+};
+
+// Launch pooling of up to two jobs (same dtype and dim) as one grid.
+cudaError_t launch_pool(int dtype, int dim, int seq_len, int block, const PoolJob* jobs,
+                        int njobs, cudaStream_t stream);
+
+struct SelectArgs {
+  const float* qc;   // [Hs, NB, ds]
+  const float* kc;   // [Hkv, NB, ds]
+  const float* kr;   // [Hkv, NB] or nullptr
+  int32_t* idx;      // [Hs, NB, kmax]
+  int32_t* cnt;      // [Hs, NB]
+  uint8_t* flags;    // [Hs, NB] or nullptr
+  int n_sel_heads;   // Hs
+  int kv_div;        // selection head hs scores against kv head hs / kv_div
+  int nb;
+  int ds;
+  int kmax;
+  int mode;          // SBSA_TOPK | SBSA_CUMMASS
+  int top_k;
+  float mass;
+  int gate;
+  float margin;
+  int rescue;
+  float tau;
+  float score_scale;
+  int* status;
+};
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+
+struct AttendArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  const int32_t* idx;
+  const int32_t* cnt;
+  int hq, hkv, n, d, block, dtype, group_shared, kmax;
+  float sm_scale;
+  int* status;
+};
+
+// Returns an SBSA_* code (SBSA_ERR_CUDA on launch/driver failure).
+int launch_attend(const AttendArgs& a, cudaStream_t stream);
+
+// One CTA waiting on an mbarrier that never completes, through the bounded
+// wait of the pipelines; records SBSA_ERR_TIMEOUT when the limit expires.
+cudaError_t launch_wait_probe(uint64_t timeout_ns, int* status, cudaStream_t stream);
+
+// Device status word of the current device (recorded by kernels).
+int* device_status_ptr();
+
+}  // namespace sbsa

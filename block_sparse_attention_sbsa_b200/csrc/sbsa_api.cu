@@ -1,0 +1,297 @@
+// C-ABI entry points: argument validation (before any launch), workspace
+// carving, dispatch to the pooling / selection / attention launchers, and
+// the per-device status word that kernels use to report runtime errors.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "internal.h"
+
+// Written by kernels (first error wins), read and cleared by sbsa_get_status.
+__device__ int g_sbsa_device_status = 0;
+
+namespace sbsa {
+
+int* device_status_ptr() {
+  static std::mutex mu;
+  static int* cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_sbsa_device_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(ptr);
+  }
+  return cache[dev];
+}
+
+namespace {
+
+struct Derived {
+  int nb;           // number of blocks
+  int group;        // Hq / Hkv
+  int hs;           // selection heads
+  int ds;           // score dimension
+  int need_kmax;    // smallest valid max_blocks
+  float sm_scale;
+  float score_scale;
+};
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Shape/option checks shared by every entry point.
+int validate(const sbsa_params* p, Derived* d) {
+  if (!p) return SBSA_ERR_INVALID_ARG;
+  if (p->n_q_heads < 1 || p->n_kv_heads < 1 || p->n_q_heads % p->n_kv_heads != 0)
+    return SBSA_ERR_INVALID_ARG;
+  if (p->seq_len < 1) return SBSA_ERR_INVALID_ARG;
+  if (p->dtype != SBSA_BF16 && p->dtype != SBSA_FP32) return SBSA_ERR_INVALID_ARG;
+  if (p->head_dim <= 0 || p->block_size <= 0 || p->index_dim < 0) return SBSA_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return SBSA_ERR_UNSUPPORTED;
+  if (p->block_size != 64 && p->block_size != 128) return SBSA_ERR_UNSUPPORTED;
+  if (p->index_dim != 0 && p->index_dim != 64 && p->index_dim != 128) return SBSA_ERR_UNSUPPORTED;
+  if (p->select_mode != SBSA_TOPK && p->select_mode != SBSA_CUMMASS) return SBSA_ERR_INVALID_ARG;
+  if (p->select_mode == SBSA_TOPK && p->top_k < 1) return SBSA_ERR_INVALID_ARG;
+  if (p->select_mode == SBSA_CUMMASS &&
+      !(p->mass_threshold > 0.f && p->mass_threshold <= 1.f))
+    return SBSA_ERR_INVALID_ARG;
+  if (p->gate && p->select_mode != SBSA_TOPK) return SBSA_ERR_INVALID_ARG;
+  if (p->gate && !(p->gate_margin >= 0.f && std::isfinite(p->gate_margin)))
+    return SBSA_ERR_INVALID_ARG;
+  if (p->rescue && std::isnan(p->rescue_tau)) return SBSA_ERR_INVALID_ARG;
+  if (!(p->sm_scale >= 0.f) || !std::isfinite(p->sm_scale)) return SBSA_ERR_INVALID_ARG;
+  if (!(p->score_scale >= 0.f) || !std::isfinite(p->score_scale)) return SBSA_ERR_INVALID_ARG;
+  Derived o;
+  o.nb = (p->seq_len + p->block_size - 1) / p->block_size;
+  o.group = p->n_q_heads / p->n_kv_heads;
+  o.hs = p->group_shared ? p->n_kv_heads : p->n_q_heads;
+  o.ds = p->index_dim ? p->index_dim : p->head_dim;
+  if (p->select_mode == SBSA_CUMMASS || p->rescue) {
+    o.need_kmax = o.nb;
+  } else {
+    long long budget = p->gate ? 2LL * p->top_k : (long long)p->top_k;
+    if (budget > o.nb - 1) budget = o.nb - 1;
+    o.need_kmax = (int)budget + 1;
+  }
+  if (p->max_blocks < o.need_kmax) return SBSA_ERR_INVALID_ARG;
+  if ((long long)p->n_q_heads * o.nb > 0x7FFFFFFFLL) return SBSA_ERR_UNSUPPORTED;
+  o.sm_scale = p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt((float)p->head_dim);
+  o.score_scale = p->score_scale > 0.f ? p->score_scale : 1.0f / std::sqrt((float)o.ds);
+  if (d) *d = o;
+  return SBSA_OK;
+}
+
+int attend_supported(const sbsa_params* p) {
+  if (p->dtype == SBSA_FP32 && !(p->head_dim == 64 && p->block_size == 64))
+    return SBSA_ERR_UNSUPPORTED;
+  return SBSA_OK;
+}
+
+struct WsLayout {
+  size_t qc, kc, kr, idx, cnt, flags, total;
+};
+
+WsLayout layout(const sbsa_params* p, const Derived& d, bool lists) {
+  WsLayout w{};
+  size_t off = 0;
+  w.qc = off;
+  off = round_up(off + (size_t)d.hs * d.nb * d.ds * 4, 256);
+  w.kc = off;
+  off = round_up(off + (size_t)p->n_kv_heads * d.nb * d.ds * 4, 256);
+  w.kr = off;
+  off = round_up(off + (p->rescue ? (size_t)p->n_kv_heads * d.nb * 4 : 0), 256);
+  w.idx = off;
+  off = round_up(off + (lists ? (size_t)d.hs * d.nb * p->max_blocks * 4 : 0), 256);
+  w.cnt = off;
+  off = round_up(off + (lists ? (size_t)d.hs * d.nb * 4 : 0), 256);
+  w.flags = off;
+  off = round_up(off + (lists ? (size_t)d.hs * d.nb : 0), 256);
+  w.total = off;
+  return w;
+}
+
+int cuda_code(cudaError_t e) { return e == cudaSuccess ? SBSA_OK : SBSA_ERR_CUDA; }
+
+SelectArgs select_args(const sbsa_params* p, const Derived& d, const float* qc, const float* kc,
+                       const float* kr, int32_t* idx, int32_t* cnt, uint8_t* flags) {
+  SelectArgs a{};
+  a.qc = qc;
+  a.kc = kc;
+  a.kr = kr;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.flags = flags;
+  a.n_sel_heads = d.hs;
+  a.kv_div = p->group_shared ? 1 : d.group;
+  a.nb = d.nb;
+  a.ds = d.ds;
+  a.kmax = p->max_blocks;
+  a.mode = p->select_mode;
+  a.top_k = p->top_k;
+  a.mass = p->mass_threshold;
+  a.gate = p->gate ? 1 : 0;
+  a.margin = p->gate_margin;
+  a.rescue = p->rescue ? 1 : 0;
+  a.tau = p->rescue_tau;
+  a.score_scale = d.score_scale;
+  a.status = device_status_ptr();
+  return a;
+}
+
+AttendArgs attend_args(const sbsa_params* p, const Derived& d, const void* q, const void* k,
+                       const void* v, const int32_t* idx, const int32_t* cnt, void* o) {
+  AttendArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.hq = p->n_q_heads;
+  a.hkv = p->n_kv_heads;
+  a.n = p->seq_len;
+  a.d = p->head_dim;
+  a.block = p->block_size;
+  a.dtype = p->dtype;
+  a.group_shared = p->group_shared ? 1 : 0;
+  a.kmax = p->max_blocks;
+  a.sm_scale = d.sm_scale;
+  a.status = device_status_ptr();
+  return a;
+}
+
+}  // namespace
+}  // namespace sbsa
+
+using namespace sbsa;
+
+extern "C" {
+
+int sbsa_version(void) { return 100; }
+
+const char* sbsa_status_string(int code) {
+  switch (code) {
+    case SBSA_OK: return "ok";
+    case SBSA_ERR_INVALID_ARG: return "invalid argument";
+    case SBSA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case SBSA_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case SBSA_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case SBSA_ERR_TIMEOUT: return "a kernel wait timed out";
+    case SBSA_ERR_DEVICE: return "a kernel met an out-of-range list entry";
+    default: return "unknown status";
+  }
+}
+
+int sbsa_pool_blocks(const sbsa_params* p, const void* x, int n_heads, int dim, int group,
+                     float* centroids, float* radii, void* stream) {
+  if (!p || !x || !centroids) return SBSA_ERR_INVALID_ARG;
+  if (p->seq_len < 1 || p->block_size <= 0) return SBSA_ERR_INVALID_ARG;
+  if (p->dtype != SBSA_BF16 && p->dtype != SBSA_FP32) return SBSA_ERR_INVALID_ARG;
+  if (p->block_size != 64 && p->block_size != 128) return SBSA_ERR_UNSUPPORTED;
+  if (n_heads < 1 || group < 1 || n_heads % group != 0) return SBSA_ERR_INVALID_ARG;
+  if (dim != 64 && dim != 128) return SBSA_ERR_UNSUPPORTED;
+  if (radii && group != 1) return SBSA_ERR_INVALID_ARG;
+  if (!aligned16(x)) return SBSA_ERR_INVALID_ARG;
+  PoolJob job{x, n_heads, group, centroids, radii};
+  return cuda_code(launch_pool(p->dtype, dim, p->seq_len, p->block_size, &job, 1,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+int sbsa_select(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
+                void* stream) {
+  Derived d;
+  int rc = validate(p, &d);
+  if (rc) return rc;
+  if (!q_cent || !k_cent || !idx || !cnt) return SBSA_ERR_INVALID_ARG;
+  if (p->rescue && !k_radius) return SBSA_ERR_INVALID_ARG;
+  if (!aligned16(q_cent) || !aligned16(k_cent)) return SBSA_ERR_INVALID_ARG;
+  SelectArgs a = select_args(p, d, q_cent, k_cent, p->rescue ? k_radius : nullptr, idx, cnt,
+                             flags);
+  return cuda_code(launch_select(a, static_cast<cudaStream_t>(stream)));
+}
+
+int sbsa_attend(const sbsa_params* p, const void* q, const void* k, const void* v,
+                const int32_t* idx, const int32_t* cnt, void* o, void* stream) {
+  Derived d;
+  int rc = validate(p, &d);
+  if (rc) return rc;
+  if (!q || !k || !v || !idx || !cnt || !o) return SBSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return SBSA_ERR_INVALID_ARG;
+  rc = attend_supported(p);
+  if (rc) return rc;
+  return launch_attend(attend_args(p, d, q, k, v, idx, cnt, o), static_cast<cudaStream_t>(stream));
+}
+
+size_t sbsa_prefill_workspace_bytes(const sbsa_params* p) {
+  Derived d;
+  if (validate(p, &d) != SBSA_OK) return 0;
+  return layout(p, d, true).total;
+}
+
+int sbsa_prefill(const sbsa_params* p, const void* q, const void* k, const void* v,
+                 const void* q_idx, const void* k_idx, void* o, void* workspace,
+                 size_t ws_bytes, int32_t* idx_out, int32_t* cnt_out, uint8_t* flags_out,
+                 void* stream) {
+  Derived d;
+  int rc = validate(p, &d);
+  if (rc) return rc;
+  if (!q || !k || !v || !o) return SBSA_ERR_INVALID_ARG;
+  if (p->index_dim && (!q_idx || !k_idx)) return SBSA_ERR_INVALID_ARG;
+  if ((idx_out == nullptr) != (cnt_out == nullptr)) return SBSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SBSA_ERR_INVALID_ARG;
+  if (p->index_dim && (!aligned16(q_idx) || !aligned16(k_idx))) return SBSA_ERR_INVALID_ARG;
+  rc = attend_supported(p);
+  if (rc) return rc;
+  const bool lists_in_ws = idx_out == nullptr;
+  WsLayout w = layout(p, d, lists_in_ws);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < w.total)
+    return SBSA_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  float* qc = reinterpret_cast<float*>(ws + w.qc);
+  float* kc = reinterpret_cast<float*>(ws + w.kc);
+  float* kr = p->rescue ? reinterpret_cast<float*>(ws + w.kr) : nullptr;
+  int32_t* idx = lists_in_ws ? reinterpret_cast<int32_t*>(ws + w.idx) : idx_out;
+  int32_t* cnt = lists_in_ws ? reinterpret_cast<int32_t*>(ws + w.cnt) : cnt_out;
+  uint8_t* flags = flags_out ? flags_out
+                             : (lists_in_ws ? reinterpret_cast<uint8_t*>(ws + w.flags) : nullptr);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* xs_k = p->index_dim ? k_idx : k;
+  const void* xs_q = p->index_dim ? q_idx : q;
+  PoolJob jobs[2] = {
+      {xs_k, p->n_kv_heads, 1, kc, kr},
+      {xs_q, p->n_q_heads, p->group_shared ? d.group : 1, qc, nullptr},
+  };
+  rc = cuda_code(launch_pool(p->dtype, d.ds, p->seq_len, p->block_size, jobs, 2, s));
+  if (rc) return rc;
+  rc = cuda_code(launch_select(select_args(p, d, qc, kc, kr, idx, cnt, flags), s));
+  if (rc) return rc;
+  return launch_attend(attend_args(p, d, q, k, v, idx, cnt, o), s);
+}
+
+int sbsa_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns < 1000ull) timeout_ns = 1000ull;
+  if (timeout_ns > 10000000000ull) timeout_ns = 10000000000ull;
+  return cuda_code(launch_wait_probe(timeout_ns, device_status_ptr(),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int sbsa_get_status(void* stream, int* device_status) {
+  if (!device_status) return SBSA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SBSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_sbsa_device_status, sizeof(int)) != cudaSuccess)
+    return SBSA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_sbsa_device_status, &zero, sizeof(int)) != cudaSuccess)
+    return SBSA_ERR_CUDA;
+  *device_status = v;
+  return SBSA_OK;
+}
+
+}  // extern "C"

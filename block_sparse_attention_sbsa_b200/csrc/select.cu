@@ -1,0 +1,460 @@
+// Block selection: pair scores, base branch (top-k, gated top-k or
+// cumulative mass), rescue branch, union with the diagonal block, ascending
+// lists with -1 padding.
+//
+// "Uncertainty-gated selection for block-sparse attention", technical
+// summary, Metodologia: step 1 block scores from a pooling backbone, step 2
+// top-k per query tile giving kv_idx, steps 3-5 a near tie at the top-k cut
+// expands the tile's budget to rho*k (rho = 2) with sentinel padding so the
+// dispatch shape stays uniform.  The gap form of the gate used here: fire
+// when s_(k) - s_(k+1) < margin * std of the row's candidate scores.
+// "RBS-Attention", method paragraph: base branch on centroid relevance and a
+// rescue branch through the block radius, each with its own threshold, masks
+// united.  "MiniMax presenta MSA": one selection per GQA group.
+//
+// Layout of one CTA: R consecutive query blocks of one selection head.
+// Phase 1 computes their scores against every earlier key block into shared
+// memory (fp32 FMA, key-centroid chunks staged in shared memory so each
+// centroid is read from L2 once per CTA).  Phase 2 gives each row to a warp:
+// exact radix selection on order-preserving 32-bit keys (ties resolved by the
+// lower block id), 64-bit fixed-point mass histograms for the cumulative-mass
+// rule (deterministic sums), double-precision mean/std for the gate, then a
+// ballot compaction that emits the ascending list.
+#include <cstdint>
+
+#include "internal.h"
+
+namespace sbsa {
+namespace {
+
+constexpr int kSelThreads = 256;
+constexpr int kWarps = kSelThreads / 32;
+constexpr int kJC = 128;  // candidate key blocks per scoring chunk
+
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// Order-preserving map of a float onto uint32 (larger float -> larger key);
+// -0 is folded onto +0 so equal scores give equal keys.
+__device__ __forceinline__ uint32_t fkey(float f) {
+  if (f == 0.0f) f = 0.0f;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_float(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(u);
+}
+
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_max_u(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// Key of descending rank `want` (0-based) among fkey(s[0..n)).  *n_gt gets
+// the number of keys strictly greater, *n_eq the number equal to it.
+__device__ uint32_t radix_select(const float* s, int n, int want, uint32_t* hist, int* n_gt,
+                                 int* n_eq) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, pmask = 0;
+  uint32_t rank = (uint32_t)want, above = 0, eq = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int base = 0; base < n; base += 32) {
+      const int j = base + lane;
+      const bool in = j < n;
+      const uint32_t u = in ? fkey(s[j]) : 0u;
+      const bool match = in && ((u & pmask) == prefix);
+      const uint32_t bin = (u >> shift) & 0xFFu;
+      const unsigned act = __ballot_sync(0xFFFFFFFFu, match);
+      if (match) {
+        const unsigned peers = __match_any_sync(act, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      }
+    }
+    __syncwarp();
+    // lane L owns bins 255-8L ... 255-8L-7, i.e. descending order by lane
+    uint32_t c[8], tot = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      c[t] = hist[255 - 8 * lane - t];
+      tot += c[t];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - tot;
+    const bool mine = excl <= rank && rank < incl;
+    const int src = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
+    uint32_t sel_bin = 0, sel_above = 0, sel_cnt = 0;
+    if (lane == src) {
+      uint32_t run = excl;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (sel_cnt == 0 && rank < run + c[t]) {
+          sel_bin = 255 - 8 * lane - t;
+          sel_above = run;
+          sel_cnt = c[t];
+        }
+        run += c[t];
+      }
+    }
+    sel_bin = __shfl_sync(0xFFFFFFFFu, sel_bin, src);
+    sel_above = __shfl_sync(0xFFFFFFFFu, sel_above, src);
+    sel_cnt = __shfl_sync(0xFFFFFFFFu, sel_cnt, src);
+    prefix |= sel_bin << shift;
+    pmask |= 0xFFu << shift;
+    rank -= sel_above;
+    above += sel_above;
+    eq = sel_cnt;
+    __syncwarp();
+  }
+  *n_gt = (int)above;
+  *n_eq = (int)eq;
+  return prefix;
+}
+
+// Fixed-point probability of a candidate: softmax weight scaled by 2^60.
+__device__ __forceinline__ uint64_t mass_weight(float s, float smax, double wscale) {
+  const float e = __expf(s - smax);
+  return (uint64_t)__double2ull_rn((double)e * wscale);
+}
+
+// Key v* of the candidate at which the score-ranked prefix mass first
+// reaches `target` (fixed point); *w_gt = mass of the keys strictly above v*.
+__device__ uint32_t radix_select_mass(const float* s, int n, float smax, double wscale,
+                                      uint64_t target, unsigned long long* hist,
+                                      uint64_t* w_gt) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, pmask = 0;
+  uint64_t above = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0ull;
+    __syncwarp();
+    for (int base = 0; base < n; base += 32) {
+      const int j = base + lane;
+      const bool in = j < n;
+      const float sv = in ? s[j] : 0.f;
+      const uint32_t u = in ? fkey(sv) : 0u;
+      const bool match = in && ((u & pmask) == prefix);
+      if (match) {
+        const uint64_t w = mass_weight(sv, smax, wscale);
+        if (w) atomicAdd(&hist[(u >> shift) & 0xFFu], (unsigned long long)w);
+      }
+    }
+    __syncwarp();
+    uint64_t c[8], tot = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      c[t] = hist[255 - 8 * lane - t];
+      tot += c[t];
+    }
+    uint64_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint64_t excl = incl - tot;
+    const uint64_t need = target - above;  // > 0 by construction
+    const bool mine = excl < need && need <= incl;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, mine);
+    const int src = bal ? __ffs(bal) - 1 : 31;
+    uint32_t sel_bin = 0;
+    uint64_t sel_above = 0;
+    if (lane == src) {
+      uint64_t run = excl;
+      bool done = false;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (!done && (need <= run + c[t] || (bal == 0 && t == 7))) {
+          sel_bin = 255 - 8 * lane - t;
+          sel_above = run;
+          done = true;
+        }
+        if (!done) run += c[t];
+      }
+    }
+    sel_bin = __shfl_sync(0xFFFFFFFFu, sel_bin, src);
+    sel_above = __shfl_sync(0xFFFFFFFFu, sel_above, src);
+    prefix |= sel_bin << shift;
+    pmask |= 0xFFu << shift;
+    above += sel_above;
+    __syncwarp();
+  }
+  *w_gt = above;
+  return prefix;
+}
+
+template <int DS, int R>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_constant__ SelectArgs a,
+                                                            int score_stride) {
+  static_assert(R % 2 == 0 && R <= 8, "rows per CTA");
+  constexpr int CS = DS + 4;  // padded centroid row stride (floats)
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* qs = reinterpret_cast<float*>(smem_raw);       // [R][DS]
+  float* cs = qs + R * DS;                              // [kJC][CS]  (phase 1)
+  float* sc = cs + kJC * CS;                            // [R][score_stride]
+  unsigned char* hist_base = reinterpret_cast<unsigned char*>(cs);  // phase 2 reuse
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int nrc = (a.nb + R - 1) / R;
+  const int rc = nrc - 1 - (int)(blockIdx.x / a.n_sel_heads);  // longest rows first
+  const int hs = (int)(blockIdx.x % a.n_sel_heads);
+  const int i0 = rc * R;
+  const int rows = min(R, a.nb - i0);
+  const int g = hs / a.kv_div;
+  const int jend = i0 + rows - 1;  // candidates needed: j < jend
+
+  for (int e = tid; e < R * DS; e += kSelThreads) {
+    const int r = e / DS;
+    qs[e] = (r < rows) ? a.qc[((size_t)hs * a.nb + i0 + r) * DS + (e % DS)] : 0.f;
+  }
+
+  // ---- phase 1: scores ----
+  constexpr int RH = R / 2;
+  const int tj = tid % kJC;
+  const int th = tid / kJC;
+  const float* kc = a.kc + (size_t)g * a.nb * DS;
+  for (int j0 = 0; j0 < jend; j0 += kJC) {
+    __syncthreads();
+    for (int e = tid * 4; e < kJC * DS; e += kSelThreads * 4) {
+      const int jj = e / DS, col = e % DS;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + jj < jend) v = *reinterpret_cast<const float4*>(kc + (size_t)(j0 + jj) * DS + col);
+      *reinterpret_cast<float4*>(cs + jj * CS + col) = v;
+    }
+    __syncthreads();
+    float acc[RH];
+#pragma unroll
+    for (int r = 0; r < RH; ++r) acc[r] = 0.f;
+    const float* crow = cs + tj * CS;
+    const float* qrow = qs + th * RH * DS;
+#pragma unroll 4
+    for (int k = 0; k < DS; k += 4) {
+      const float4 c4 = *reinterpret_cast<const float4*>(crow + k);
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        const float4 q4 = *reinterpret_cast<const float4*>(qrow + r * DS + k);
+        acc[r] = fmaf(q4.x, c4.x, acc[r]);
+        acc[r] = fmaf(q4.y, c4.y, acc[r]);
+        acc[r] = fmaf(q4.z, c4.z, acc[r]);
+        acc[r] = fmaf(q4.w, c4.w, acc[r]);
+      }
+    }
+    const int j = j0 + tj;
+    if (j < jend) {
+#pragma unroll
+      for (int r = 0; r < RH; ++r) sc[(th * RH + r) * score_stride + j] = acc[r] * a.score_scale;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 2: one warp per row ----
+  unsigned long long* hist64 =
+      reinterpret_cast<unsigned long long*>(hist_base) + (size_t)warp * 256;
+  uint32_t* hist32 = reinterpret_cast<uint32_t*>(hist64);
+  const unsigned lt_mask = (1u << lane) - 1u;
+
+  for (int r = warp; r < rows; r += kWarps) {
+    const int i = i0 + r;
+    const int n = i;  // candidates j < i
+    const float* s = sc + (size_t)r * score_stride;
+    int32_t* out = a.idx + ((size_t)hs * a.nb + i) * a.kmax;
+
+    // threshold key and how many tied keys to take (in ascending id order)
+    uint32_t vkey = 0xFFFFFFFFu;
+    int take_eq = 0;
+    bool select_all = false;
+    uint8_t flag = 0;
+    if (a.mode == SBSA_TOPK) {
+      int kk = a.top_k;
+      if (n <= kk) {
+        select_all = true;
+      } else {
+        int n_gt, n_eq;
+        vkey = radix_select(s, n, kk - 1, hist32, &n_gt, &n_eq);
+        take_eq = kk - n_gt;
+        if (a.gate) {
+          // s_(k) and s_(k+1); population std of the candidates (double)
+          const float sk = key_float(vkey);
+          float sk1;
+          if (n_gt + n_eq >= kk + 1) {
+            sk1 = sk;
+          } else {
+            uint32_t below = 0;
+            for (int j = lane; j < n; j += 32) {
+              const uint32_t u = fkey(s[j]);
+              if (u < vkey) below = max(below, u);
+            }
+            sk1 = key_float(warp_max_u(below));
+          }
+          double sum = 0.0;
+          for (int j = lane; j < n; j += 32) sum += (double)s[j];
+          const double mean = warp_sum_d(sum) / (double)n;
+          double ss = 0.0;
+          for (int j = lane; j < n; j += 32) {
+            const double dlt = (double)s[j] - mean;
+            ss += dlt * dlt;
+          }
+          const double sd = sqrt(warp_sum_d(ss) / (double)n);
+          const double gap = (double)sk - (double)sk1;
+          if (gap < (double)a.margin * sd) {
+            flag |= 1;
+            kk = 2 * a.top_k;
+            if (n <= kk) {
+              select_all = true;
+            } else {
+              vkey = radix_select(s, n, kk - 1, hist32, &n_gt, &n_eq);
+              take_eq = kk - n_gt;
+            }
+          }
+        }
+      }
+    } else {  // SBSA_CUMMASS
+      if (n == 0) {
+        select_all = true;
+      } else {
+        float m = -INFINITY;
+        for (int j = lane; j < n; j += 32) m = fmaxf(m, s[j]);
+        m = warp_max_f(m);
+        double z = 0.0;
+        for (int j = lane; j < n; j += 32) z += (double)__expf(s[j] - m);
+        z = warp_sum_d(z);
+        const double wscale = 1152921504606846976.0 / z;  // 2^60 / Z
+        uint64_t wtot = 0;
+        for (int j = lane; j < n; j += 32) wtot += mass_weight(s[j], m, wscale);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) wtot += __shfl_xor_sync(0xFFFFFFFFu, wtot, o);
+        double tgt_d = ceil((double)a.mass * 1152921504606846976.0);
+        uint64_t target = (uint64_t)tgt_d;
+        if (target > wtot) target = wtot;
+        if (target == 0) target = 1;
+        if (wtot == 0) {
+          select_all = true;
+        } else {
+          uint64_t w_gt;
+          vkey = radix_select_mass(s, n, m, wscale, target, hist64, &w_gt);
+          const uint64_t w_one = mass_weight(key_float(vkey), m, wscale);
+          // tied keys all carry w_one; take the fewest that reach the target
+          uint64_t t = w_one ? (target - w_gt + w_one - 1) / w_one : 1;
+          if (t < 1) t = 1;
+          if (t > (uint64_t)n) t = (uint64_t)n;
+          take_eq = (int)t;
+        }
+      }
+    }
+
+    // rescue bound scale: |q| * score_scale
+    float qn_s = 0.f;
+    if (a.rescue) {
+      const float* qv = qs + r * DS;
+      float q2 = 0.f;
+      for (int c = lane; c < DS; c += 32) q2 = fmaf(qv[c], qv[c], q2);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) q2 += __shfl_xor_sync(0xFFFFFFFFu, q2, o);
+      qn_s = sqrtf(q2) * a.score_scale;
+    }
+    const float* kr = a.rescue ? a.kr + (size_t)g * a.nb : nullptr;
+
+    // ---- compaction: ascending ids, then the diagonal, then -1 ----
+    int written = 0, tie_seen = 0;
+    bool rescued_extra = false;
+    for (int base = 0; base < n; base += 32) {
+      const int j = base + lane;
+      const bool in = j < n;
+      bool sel = false, eqk = false, basesel = false;
+      if (in) {
+        if (select_all) {
+          basesel = true;
+        } else {
+          const uint32_t u = fkey(s[j]);
+          basesel = u > vkey;
+          eqk = (u == vkey);
+        }
+      }
+      const unsigned eqmask = __ballot_sync(0xFFFFFFFFu, eqk);
+      if (eqk) basesel = (tie_seen + __popc(eqmask & lt_mask)) < take_eq;
+      tie_seen += __popc(eqmask);
+      sel = basesel;
+      if (in && a.rescue) {
+        const float ub = fmaf(qn_s, kr[j], s[j]);
+        if (ub > a.tau) {
+          sel = true;
+          if (!basesel) rescued_extra = true;
+        }
+      }
+      const unsigned selmask = __ballot_sync(0xFFFFFFFFu, sel);
+      const int pos = written + __popc(selmask & lt_mask);
+      if (sel && pos < a.kmax - 1) out[pos] = j;
+      written += __popc(selmask);
+    }
+    if (__any_sync(0xFFFFFFFFu, rescued_extra)) flag |= 2;
+    if (written > a.kmax - 1) {
+      if (lane == 0) record_status(a.status, SBSA_ERR_DEVICE);
+      written = a.kmax - 1;
+    }
+    if (lane == 0) {
+      out[written] = i;
+      a.cnt[(size_t)hs * a.nb + i] = written + 1;
+      if (a.flags) a.flags[(size_t)hs * a.nb + i] = flag;
+    }
+    for (int p = written + 1 + lane; p < a.kmax; p += 32) out[p] = -1;
+    __syncwarp();
+  }
+}
+
+template <int DS, int R>
+cudaError_t launch_rows(const SelectArgs& a, cudaStream_t stream) {
+  const int stride = (a.nb + 3) & ~3;
+  const size_t smem = (size_t)(R * DS + kJC * (DS + 4) + R * stride) * sizeof(float);
+  const size_t hist_need = (size_t)kWarps * 256 * 8;
+  if (hist_need > (size_t)kJC * (DS + 4) * sizeof(float)) return cudaErrorInvalidValue;
+  auto kern = select_kernel<DS, R>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long nrc = (a.nb + R - 1) / R;
+  const long long grid = nrc * a.n_sel_heads;
+  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  kern<<<(unsigned)grid, kSelThreads, smem, stream>>>(a, stride);
+  return cudaGetLastError();
+}
+
+template <int DS>
+cudaError_t launch_ds(const SelectArgs& a, cudaStream_t stream) {
+  // rows per CTA: as many as the score rows fit next to the centroid chunk
+  const size_t fixed = (size_t)kJC * (DS + 4) * 4;
+  const size_t budget = 220 * 1024;
+  const size_t row = (size_t)((a.nb + 3) & ~3) * 4 + DS * 4;
+  if (fixed + 8 * row <= budget) return launch_rows<DS, 8>(a, stream);
+  if (fixed + 4 * row <= budget) return launch_rows<DS, 4>(a, stream);
+  if (fixed + 2 * row <= budget) return launch_rows<DS, 2>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
+  return a.ds == 128 ? launch_ds<128>(a, stream) : launch_ds<64>(a, stream);
+}
+
+}  // namespace sbsa

@@ -1,0 +1,335 @@
+"""ctypes binding over libsbsa.so (argument marshalling only).
+
+Every function takes torch CUDA tensors (PyTorch provides device memory and
+the stream), passes raw pointers and sizes to the C ABI declared in
+include/sbsa.h, and raises on a non-zero status.  All compute runs in the
+library's CUDA kernels; there is no fallback of any kind: if the library is
+missing or fails to load, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsbsa.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
+BF16, FP32 = 0, 1
+TOPK, CUMMASS = 0, 1
+FLAG_GATE, FLAG_RESCUE = 1, 2
+
+SYMBOLS = ["sbsa_pool_blocks", "sbsa_select", "sbsa_attend", "sbsa_prefill",
+           "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string",
+           "sbsa_version", "sbsa_debug_wait_timeout"]
+
+
+class SbsaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (code {code})")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [
+        ("n_q_heads", ctypes.c_int),
+        ("n_kv_heads", ctypes.c_int),
+        ("seq_len", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("block_size", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+        ("select_mode", ctypes.c_int),
+        ("group_shared", ctypes.c_int),
+        ("index_dim", ctypes.c_int),
+        ("top_k", ctypes.c_int),
+        ("mass_threshold", ctypes.c_float),
+        ("rescue", ctypes.c_int),
+        ("rescue_tau", ctypes.c_float),
+        ("gate", ctypes.c_int),
+        ("gate_margin", ctypes.c_float),
+        ("max_blocks", ctypes.c_int),
+        ("sm_scale", ctypes.c_float),
+        ("score_scale", ctypes.c_float),
+    ]
+
+    @property
+    def n_blocks(self) -> int:
+        return (self.seq_len + self.block_size - 1) // self.block_size
+
+    @property
+    def n_sel_heads(self) -> int:
+        return self.n_kv_heads if self.group_shared else self.n_q_heads
+
+    @property
+    def score_dim(self) -> int:
+        return self.index_dim if self.index_dim else self.head_dim
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_sbsa_b200.build`"
+            " (there is no non-CUDA fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(Params)
+    vp, i32p, f32p, u8p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    ci = ctypes.c_int
+    lib.sbsa_pool_blocks.argtypes = [P, vp, ci, ci, ci, f32p, f32p, vp]
+    lib.sbsa_select.argtypes = [P, f32p, f32p, f32p, i32p, i32p, u8p, vp]
+    lib.sbsa_attend.argtypes = [P, vp, vp, vp, i32p, i32p, vp, vp]
+    lib.sbsa_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i32p, i32p, u8p, vp]
+    lib.sbsa_prefill_workspace_bytes.argtypes = [P]
+    lib.sbsa_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.sbsa_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.sbsa_status_string.argtypes = [ci]
+    lib.sbsa_status_string.restype = ctypes.c_char_p
+    lib.sbsa_version.argtypes = []
+    lib.sbsa_debug_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    for name in ["sbsa_pool_blocks", "sbsa_select", "sbsa_attend", "sbsa_prefill",
+                 "sbsa_get_status", "sbsa_version", "sbsa_debug_wait_timeout"]:
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def status_string(code: int) -> str:
+    return lib.sbsa_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise SbsaError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def make_params(*, n_q_heads, n_kv_heads, seq_len, head_dim, block_size, dtype="bf16",
+                select_mode="topk", top_k=0, mass_threshold=0.0, rescue_tau=None,
+                gate_margin=None, group_shared=False, index_dim=0, max_blocks=None,
+                sm_scale=0.0, score_scale=0.0) -> Params:
+    p = Params()
+    p.n_q_heads, p.n_kv_heads, p.seq_len = n_q_heads, n_kv_heads, seq_len
+    p.head_dim, p.block_size = head_dim, block_size
+    p.dtype = {"bf16": BF16, "fp32": FP32}[dtype] if isinstance(dtype, str) else int(dtype)
+    p.select_mode = {"topk": TOPK, "cummass": CUMMASS}[select_mode] if isinstance(select_mode, str) else int(select_mode)
+    p.group_shared = 1 if group_shared else 0
+    p.index_dim = index_dim
+    p.top_k = top_k
+    p.mass_threshold = mass_threshold
+    p.rescue = 0 if rescue_tau is None else 1
+    p.rescue_tau = 0.0 if rescue_tau is None else float(rescue_tau)
+    p.gate = 0 if gate_margin is None else 1
+    p.gate_margin = 0.0 if gate_margin is None else float(gate_margin)
+    nb = (seq_len + block_size - 1) // block_size
+    if max_blocks is None:
+        if p.select_mode == CUMMASS or p.rescue:
+            max_blocks = nb
+        else:
+            budget = 2 * top_k if p.gate else top_k
+            max_blocks = min(budget, nb - 1) + 1
+    p.max_blocks = max_blocks
+    p.sm_scale = sm_scale
+    p.score_scale = score_scale
+    return p
+
+
+def params_for(w) -> Params:
+    """Parameters of a workload description (block_sparse_attention_sbsa_b200.workloads)."""
+    return make_params(n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, seq_len=w.seq_len,
+                       head_dim=w.head_dim, block_size=w.block_size, dtype=w.dtype,
+                       select_mode=w.select_mode, top_k=w.top_k,
+                       mass_threshold=w.mass_threshold, rescue_tau=w.rescue_tau,
+                       gate_margin=w.gate_margin, group_shared=w.group_shared,
+                       index_dim=w.index_dim, max_blocks=w.max_blocks)
+
+
+_TORCH_DT = {BF16: torch.bfloat16, FP32: torch.float32}
+
+
+def pool_blocks(p: Params, x: torch.Tensor, group: int = 1, radius: bool = False, stream=None):
+    """Centroids [H/group, NB, dim] (and radii [H, NB]) of x [H, N, dim]."""
+    _need(x, "x", _TORCH_DT[p.dtype])
+    h, n, dim = x.shape
+    if n != p.seq_len:
+        raise ValueError("x.shape[1] must equal seq_len")
+    nb = p.n_blocks
+    cent = torch.empty(h // group, nb, dim, device=x.device, dtype=torch.float32)
+    rad = torch.empty(h, nb, device=x.device, dtype=torch.float32) if radius else None
+    _check(lib.sbsa_pool_blocks(ctypes.byref(p), _ptr(x), h, dim, group, _ptr(cent), _ptr(rad),
+                                _stream(stream)), "sbsa_pool_blocks")
+    return cent, rad
+
+
+def select(p: Params, q_cent: torch.Tensor, k_cent: torch.Tensor,
+           k_radius: Optional[torch.Tensor] = None, stream=None, with_flags: bool = True):
+    """Block lists (idx [Hs, NB, Kmax], cnt [Hs, NB], flags [Hs, NB])."""
+    nb, hs, ds = p.n_blocks, p.n_sel_heads, p.score_dim
+    _need(q_cent, "q_cent", torch.float32, (hs, nb, ds))
+    _need(k_cent, "k_cent", torch.float32, (p.n_kv_heads, nb, ds))
+    if p.rescue:
+        _need(k_radius, "k_radius", torch.float32, (p.n_kv_heads, nb))
+    dev = q_cent.device
+    idx = torch.empty(hs, nb, p.max_blocks, device=dev, dtype=torch.int32)
+    cnt = torch.empty(hs, nb, device=dev, dtype=torch.int32)
+    flags = torch.empty(hs, nb, device=dev, dtype=torch.uint8) if with_flags else None
+    _check(lib.sbsa_select(ctypes.byref(p), _ptr(q_cent), _ptr(k_cent),
+                           _ptr(k_radius) if p.rescue else None, _ptr(idx), _ptr(cnt),
+                           _ptr(flags), _stream(stream)), "sbsa_select")
+    return idx, cnt, flags
+
+
+def attend(p: Params, q, k, v, idx, cnt, out=None, stream=None):
+    """O [Hq, N, d] of attention restricted to the listed blocks."""
+    dt = _TORCH_DT[p.dtype]
+    _need(q, "q", dt, (p.n_q_heads, p.seq_len, p.head_dim))
+    _need(k, "k", dt, (p.n_kv_heads, p.seq_len, p.head_dim))
+    _need(v, "v", dt, (p.n_kv_heads, p.seq_len, p.head_dim))
+    _need(idx, "idx", torch.int32, (p.n_sel_heads, p.n_blocks, p.max_blocks))
+    _need(cnt, "cnt", torch.int32, (p.n_sel_heads, p.n_blocks))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", dt, q.shape)
+    _check(lib.sbsa_attend(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt),
+                           _ptr(out), _stream(stream)), "sbsa_attend")
+    return out
+
+
+def workspace_bytes(p: Params) -> int:
+    n = lib.sbsa_prefill_workspace_bytes(ctypes.byref(p))
+    if n == 0:
+        raise SbsaError(ERR_INVALID_ARG, "sbsa_prefill_workspace_bytes")
+    return int(n)
+
+
+class Prefill:
+    """Reusable prefill call: owns the workspace and optional list outputs so
+    repeated calls allocate nothing."""
+
+    def __init__(self, p: Params, device="cuda", keep_lists: bool = True):
+        self.p = p
+        self.ws = torch.empty(workspace_bytes(p), device=device, dtype=torch.uint8)
+        nb, hs = p.n_blocks, p.n_sel_heads
+        if keep_lists:
+            self.idx = torch.empty(hs, nb, p.max_blocks, device=device, dtype=torch.int32)
+            self.cnt = torch.empty(hs, nb, device=device, dtype=torch.int32)
+            self.flags = torch.empty(hs, nb, device=device, dtype=torch.uint8)
+        else:
+            self.idx = self.cnt = self.flags = None
+
+    def __call__(self, q, k, v, q_idx=None, k_idx=None, out=None, stream=None):
+        p = self.p
+        dt = _TORCH_DT[p.dtype]
+        _need(q, "q", dt, (p.n_q_heads, p.seq_len, p.head_dim))
+        _need(k, "k", dt, (p.n_kv_heads, p.seq_len, p.head_dim))
+        _need(v, "v", dt, (p.n_kv_heads, p.seq_len, p.head_dim))
+        if p.index_dim:
+            _need(q_idx, "q_idx", dt, (p.n_q_heads, p.seq_len, p.index_dim))
+            _need(k_idx, "k_idx", dt, (p.n_kv_heads, p.seq_len, p.index_dim))
+        if out is None:
+            out = torch.empty_like(q)
+        _check(lib.sbsa_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(q_idx) if p.index_dim else None,
+                                _ptr(k_idx) if p.index_dim else None, _ptr(out), _ptr(self.ws),
+                                self.ws.numel(), _ptr(self.idx), _ptr(self.cnt), _ptr(self.flags),
+                                _stream(stream)), "sbsa_prefill")
+        return out
+
+
+def prefill(p: Params, q, k, v, q_idx=None, k_idx=None, stream=None):
+    """One-shot prefill; returns (O, idx, cnt, flags)."""
+    call = Prefill(p, device=q.device)
+    out = call(q, k, v, q_idx, k_idx, stream=stream)
+    return out, call.idx, call.cnt, call.flags
+
+
+def debug_wait_timeout(timeout_ns: int, stream=None):
+    """Launch the bounded-wait probe (see include/sbsa.h)."""
+    _check(lib.sbsa_debug_wait_timeout(int(timeout_ns), _stream(stream)),
+           "sbsa_debug_wait_timeout")
+
+
+def get_status(stream=None) -> int:
+    """Synchronise the stream and read/clear the device status word."""
+    st = ctypes.c_int(0)
+    _check(lib.sbsa_get_status(_stream(stream), ctypes.byref(st)), "sbsa_get_status")
+    return st.value
+
+
+class Staged:
+    """The prefill as its separate C-ABI stages on preallocated buffers:
+    pool keys (+ radii), pool queries, select, attend.  Each method is one
+    library call and allocates nothing; the kernels are the ones
+    sbsa_prefill launches (which merges the two pooling jobs into one grid)."""
+
+    def __init__(self, p: Params, device="cuda"):
+        self.p = p
+        nb, hs, ds, hk = p.n_blocks, p.n_sel_heads, p.score_dim, p.n_kv_heads
+        f32 = dict(device=device, dtype=torch.float32)
+        self.kc = torch.empty(hk, nb, ds, **f32)
+        self.kr = torch.empty(hk, nb, **f32) if p.rescue else None
+        self.qc = torch.empty(hs, nb, ds, **f32)
+        self.idx = torch.empty(hs, nb, p.max_blocks, device=device, dtype=torch.int32)
+        self.cnt = torch.empty(hs, nb, device=device, dtype=torch.int32)
+        self.flags = torch.empty(hs, nb, device=device, dtype=torch.uint8)
+        self._p = ctypes.byref(p)
+
+    def pool(self, q_src, k_src, stream=None):
+        p, s = self.p, _stream(stream)
+        ds = p.score_dim
+        grp = (p.n_q_heads // p.n_kv_heads) if p.group_shared else 1
+        _check(lib.sbsa_pool_blocks(self._p, _ptr(k_src), p.n_kv_heads, ds, 1, _ptr(self.kc),
+                                    _ptr(self.kr), s), "sbsa_pool_blocks")
+        _check(lib.sbsa_pool_blocks(self._p, _ptr(q_src), p.n_q_heads, ds, grp, _ptr(self.qc),
+                                    None, s), "sbsa_pool_blocks")
+
+    def select(self, stream=None):
+        _check(lib.sbsa_select(self._p, _ptr(self.qc), _ptr(self.kc), _ptr(self.kr),
+                               _ptr(self.idx), _ptr(self.cnt), _ptr(self.flags),
+                               _stream(stream)), "sbsa_select")
+
+    def attend(self, q, k, v, out, stream=None):
+        _check(lib.sbsa_attend(self._p, _ptr(q), _ptr(k), _ptr(v), _ptr(self.idx),
+                               _ptr(self.cnt), _ptr(out), _stream(stream)), "sbsa_attend")
+
+
+def attended_pairs(p: Params, cnt: torch.Tensor) -> int:
+    """Unmasked (query, key) pairs of the attention over the lists `cnt`
+    describes, assuming each list holds valid ids ending with its diagonal
+    block: full B x rows for every earlier block, the causal triangle for
+    the diagonal block."""
+    b, n, nb = p.block_size, p.seq_len, p.n_blocks
+    c = cnt.to(torch.int64).cpu()
+    rows = torch.full((nb,), b, dtype=torch.int64)
+    rows[-1] = n - (nb - 1) * b
+    diag = rows * (rows + 1) // 2
+    if p.group_shared:
+        c = c.repeat_interleave(p.n_q_heads // p.n_kv_heads, dim=0)
+    past = ((c - 1).clamp(min=0) * rows.view(1, -1) * b).sum()
+    return int(past + (diag.view(1, -1) * (c > 0)).sum())

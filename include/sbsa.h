@@ -1,0 +1,180 @@
+/*
+ * sbsa.h -- block-sparse attention prefill on NVIDIA B200 (sm_100a).
+ *
+ * A C ABI over four device stages: pool key/query blocks, select a block
+ * list per query block, attend over the listed blocks, and the whole
+ * prefill.  All tensor arguments are DEVICE pointers owned by the caller;
+ * the library never allocates, frees or retains memory between calls.
+ * Every call is asynchronous on the caller's stream (a cudaStream_t passed
+ * as `void*`; NULL means the legacy default stream) and returns a status
+ * code.  Argument errors are detected on the host before any launch; in
+ * that case nothing is enqueued.  Errors detected by a kernel (a bounded
+ * wait that expired, an index out of range) are recorded in a per-device
+ * status word read by sbsa_get_status().
+ *
+ * Sources of the operations (web pages, by title and section):
+ *   [RBS]  "RBS-Attention: un metodo de prefill disperso para modelos de
+ *          lenguaje con contexto largo" (iaonda.com), method paragraph: key
+ *          blocks summarised by a centroid and a dynamic radius; a base
+ *          branch (centroid relevance) and a rescue branch (blocks at risk
+ *          of being underestimated) each with an independent threshold;
+ *          masks united; sparse-FlashAttention-compatible prefill.
+ *   [UGS]  "Uncertainty-gated selection for block-sparse attention"
+ *          (gist.science, paper 2607.07724), technical summary,
+ *          Metodologia steps 1-5: mean-pooled block scores, per-query-tile
+ *          top-k lists kv_idx, expansion to 2k where the top-k cut is
+ *          ambiguous, sentinel padding for uniform dispatch shapes.
+ *   [MSA]  "MiniMax presenta MSA ..." (iaonda.com), "Que es MSA y como
+ *          funciona?": one top-k selection per GQA group from a light index
+ *          branch; full attention over the preselected blocks only.
+ *
+ * Layout (all tensors contiguous, batch 1, one layer):
+ *   Q  [Hq,  N, d]      K, V [Hkv, N, d]      O [Hq, N, d]
+ *   Q_idx [Hq, N, d_idx], K_idx [Hkv, N, d_idx]   (optional index tensors)
+ * Element type of Q/K/V/O and of the index tensors: p->dtype.
+ * Query head h reads kv head h / (Hq/Hkv).  Token t belongs to block t / B;
+ * NB = ceil(N / B) and the last block may be partial.
+ */
+#ifndef SBSA_H_
+#define SBSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+#define SBSA_OK 0
+#define SBSA_ERR_INVALID_ARG 1 /* null pointer, inconsistent shape or option  */
+#define SBSA_ERR_UNSUPPORTED 2 /* valid but not built: d, B, d_idx, dtype     */
+#define SBSA_ERR_WORKSPACE 3   /* workspace too small or misaligned           */
+#define SBSA_ERR_CUDA 4        /* a CUDA runtime/driver call failed           */
+#define SBSA_ERR_TIMEOUT 5     /* a kernel's bounded wait expired             */
+#define SBSA_ERR_DEVICE 6      /* a kernel met an out-of-range list entry     */
+
+/* ---- element types ---- */
+#define SBSA_BF16 0 /* bfloat16 storage, bf16 tensor-core products, fp32 accumulate */
+#define SBSA_FP32 1 /* fp32 storage, tf32 tensor-core products, fp32 accumulate     */
+
+/* ---- base-branch selection rules ---- */
+#define SBSA_TOPK 0    /* [UGS] step 2: the top_k best-scoring past blocks           */
+#define SBSA_CUMMASS 1 /* [RBS] base branch: shortest score-ranked prefix whose
+                          softmax mass over the candidates reaches mass_threshold */
+
+typedef struct sbsa_params {
+  int n_q_heads;        /* Hq >= 1                                             */
+  int n_kv_heads;       /* Hkv >= 1, divides Hq (GQA group G = Hq/Hkv)         */
+  int seq_len;          /* N >= 1                                              */
+  int head_dim;         /* d in {64, 128}                                      */
+  int block_size;       /* B in {64, 128}; query tile = key block = B tokens   */
+  int dtype;            /* SBSA_BF16 | SBSA_FP32 (fp32 attention: d = 64 only) */
+  int select_mode;      /* SBSA_TOPK | SBSA_CUMMASS                            */
+  int group_shared;     /* 0: one list per query head; 1: one per GQA group    */
+  int index_dim;        /* 0: score on Q/K; else d_idx in {64,128} of Q_idx/K_idx */
+  int top_k;            /* TOPK budget k >= 1                                  */
+  float mass_threshold; /* CUMMASS threshold in (0, 1]                         */
+  int rescue;           /* 1: unite with the rescue branch (needs radii)       */
+  float rescue_tau;     /* rescue keeps j when (q.c_j + |q| r_j)*score_scale > tau */
+  int gate;             /* 1: uncertainty gate (TOPK only)                     */
+  float gate_margin;    /* gate fires when s_(k) - s_(k+1) < margin * std(s)   */
+  int max_blocks;       /* list width Kmax; must hold the widest possible list:
+                           TOPK min(k,NB-1)+1, gated min(2k,NB-1)+1,
+                           CUMMASS or rescue NB                                */
+  float sm_scale;       /* attention logit scale; 0 => 1/sqrt(head_dim)       */
+  float score_scale;    /* block-score scale;     0 => 1/sqrt(score dim)      */
+} sbsa_params;
+
+/*
+ * sbsa_pool_blocks -- [RBS] centroid and radius of each block; [UGS] step 1
+ * mean pooling; [MSA] group-level pooled queries.
+ *   x         device [n_heads, N, dim], element type p->dtype.
+ *   group     consecutive heads averaged into one output head (1 = none);
+ *             must divide n_heads.
+ *   centroids device fp32 [n_heads/group, NB, dim]:
+ *             mean over the group's heads of each head's mean over the rows
+ *             of block j (rows t with t/B == j, t < N).
+ *   radii     device fp32 [n_heads, NB] or NULL: max_t |x_t - c_j|_2 over the
+ *             block's rows (group must be 1 when radii is given).
+ * Uses N and B from p; dim in {64, 128}.  Reads x once.
+ */
+int sbsa_pool_blocks(const sbsa_params* p, const void* x, int n_heads, int dim, int group,
+                     float* centroids, float* radii, void* stream);
+
+/*
+ * sbsa_select -- [UGS] steps 1-5 on pooled tables; [RBS] base and rescue
+ * branches with their union; [MSA] group-shared lists.
+ *   q_cent   device fp32 [Hs, NB, ds]  pooled queries, Hs = group_shared ? Hkv : Hq
+ *   k_cent   device fp32 [Hkv, NB, ds] key centroids
+ *   k_radius device fp32 [Hkv, NB] (required when p->rescue, else ignored)
+ *   idx      device int32 [Hs, NB, max_blocks] out: ascending block ids, then -1
+ *   cnt      device int32 [Hs, NB] out: number of valid ids per row
+ *   flags    device uint8 [Hs, NB] out or NULL: bit0 gate fired, bit1 rescue
+ *            added a block the base branch missed
+ * ds = index_dim if set, else head_dim.  Selection head hs scores against kv
+ * head (group_shared ? hs : hs / G).  Candidates of query block i are the
+ * blocks j < i with score s_j = (q_cent[hs,i] . k_cent[g,j]) * score_scale,
+ * ranked by score descending, lower id first on equal scores.  The diagonal
+ * block i is always appended.
+ */
+int sbsa_select(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags, void* stream);
+
+/*
+ * sbsa_attend -- [RBS] sparse prefill attention; [MSA] main branch.
+ *   q [Hq,N,d], k/v [Hkv,N,d], o [Hq,N,d]: device, element type p->dtype.
+ *   idx/cnt: lists as produced by sbsa_select (Hs rows per p->group_shared).
+ * O[h,t] = sum over u in the listed blocks of (h, t/B) with u <= t of
+ * softmax_u(Q[h,t].K[g,u] * sm_scale) V[g,u]; rows that see no key are 0.
+ * List entries outside [0, i] are skipped and reported as SBSA_ERR_DEVICE
+ * through sbsa_get_status; a repeated entry is attended twice.
+ */
+int sbsa_attend(const sbsa_params* p, const void* q, const void* k, const void* v,
+                const int32_t* idx, const int32_t* cnt, void* o, void* stream);
+
+/* Bytes of device workspace sbsa_prefill needs for these parameters
+ * (pooled tables, plus lists when the caller does not provide them).
+ * Returns 0 when p is invalid. */
+size_t sbsa_prefill_workspace_bytes(const sbsa_params* p);
+
+/*
+ * sbsa_prefill -- pool (keys and queries), select, attend, on one stream.
+ *   q_idx/k_idx: index tensors when p->index_dim != 0 (else NULL).
+ *   workspace:   device, 256-byte aligned, ws_bytes >= sbsa_prefill_workspace_bytes(p).
+ *   idx_out/cnt_out/flags_out: optional device outputs (layout of sbsa_select);
+ *   when NULL the lists live in the workspace.
+ */
+int sbsa_prefill(const sbsa_params* p, const void* q, const void* k, const void* v,
+                 const void* q_idx, const void* k_idx, void* o, void* workspace,
+                 size_t ws_bytes, int32_t* idx_out, int32_t* cnt_out, uint8_t* flags_out,
+                 void* stream);
+
+/* Synchronises `stream`, then reads and clears the current device's status
+ * word into *device_status (SBSA_OK when no kernel reported an error).
+ * Returns SBSA_ERR_CUDA when the synchronisation itself failed. */
+int sbsa_get_status(void* stream, int* device_status);
+
+/* Static description of a status code. */
+const char* sbsa_status_string(int code);
+
+/* Library ABI version (major * 100 + minor). */
+int sbsa_version(void);
+
+/*
+ * sbsa_debug_wait_timeout -- test hook for the failure path of the bounded
+ * device waits used by the kernels (no counterpart on the pages).  Launches
+ * one CTA that waits on an mbarrier nothing ever arrives on, using the same
+ * bounded-wait primitive as the attention pipeline with a limit of
+ * `timeout_ns` nanoseconds (clamped to [1 us, 10 s]); when the limit expires
+ * the kernel records SBSA_ERR_TIMEOUT in the device status word and returns.
+ * No copy or MMA is in flight, so the context stays usable.  Read the result
+ * with sbsa_get_status().
+ */
+int sbsa_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBSA_H_ */

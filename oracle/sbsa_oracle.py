@@ -240,16 +240,16 @@ def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
 # prefill; MSA: full attention over the preselected blocks)
 # --------------------------------------------------------------------------
 
-def attend_block(q, k, v, blocks, i: int, block: int, scale: float):
+def attend_block(q_rows, k, v, blocks, i: int, block: int, scale: float):
     """Output rows of query block i for one head: for each query t, softmax
     over the keys u of the listed blocks with u <= t of (q_t . k_u) * scale,
-    weighting v_u.  Rows that see no key return zeros.  q is [N, d] of the
-    query head, k and v [N, d] of its kv head."""
-    n = q.shape[0]
+    weighting v_u.  Rows that see no key return zeros.  q_rows holds the
+    query rows of block i, k and v are [N, d] of the head's kv head."""
+    n = k.shape[0]
     t_rows = np.arange(i * block, min(n, (i + 1) * block))
     u = np.concatenate([np.arange(j * block, min(n, (j + 1) * block))
                         for j in blocks]) if len(blocks) else np.zeros(0, np.int64)
-    qt = _f64(q[t_rows[0]:t_rows[-1] + 1])
+    qt = _f64(q_rows)
     out = np.zeros((len(t_rows), v.shape[1]))
     if len(u) == 0:
         return out
@@ -258,13 +258,14 @@ def attend_block(q, k, v, blocks, i: int, block: int, scale: float):
     logits = (qt @ ku.T) * scale
     visible = u[None, :] <= t_rows[:, None]
     logits = np.where(visible, logits, -np.inf)
-    for row in range(len(t_rows)):
-        if not visible[row].any():
-            continue
-        z = logits[row] - logits[row][visible[row]].max()
-        p = np.exp(z)
-        p /= p.sum()
-        out[row] = p @ vu
+    seen = visible.any(axis=1)
+    if not seen.any():
+        return out
+    rows = np.nonzero(seen)[0]
+    z = logits[rows] - logits[rows].max(axis=1, keepdims=True)
+    p = np.exp(z)                              # exp(-inf) = 0 off the mask
+    p /= p.sum(axis=1, keepdims=True)
+    out[rows] = p @ vu
     return out
 
 
@@ -283,8 +284,8 @@ def attend(q, k, v, idx, cnt, *, block: int, scale: float, group_shared: bool,
         g = h // grp
         hs = g if group_shared else h
         blocks = [int(x) for x in idx[hs, i, :cnt[hs, i]]]
-        out[h, i * block:min(n, (i + 1) * block)] = attend_block(
-            q[h], k[g], v[g], blocks, i, block, scale)
+        lo, hi = i * block, min(n, (i + 1) * block)
+        out[h, lo:hi] = attend_block(q[h, lo:hi], k[g], v[g], blocks, i, block, scale)
     return out
 
 

@@ -1,0 +1,169 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, its parameter struct matches the C layout, and argument
+errors are rejected on the host before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sbsa.h")
+
+
+@pytest.fixture(scope="module")
+def sb():
+    from block_sparse_attention_sbsa_b200 import build
+    build.build()
+    from block_sparse_attention_sbsa_b200 import sbsa
+    return sbsa
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\*]+\s+\**(sbsa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["sbsa_pool_blocks", "sbsa_select", "sbsa_attend", "sbsa_prefill",
+                     "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(sb):
+    out = subprocess.run(["nm", "-D", "--defined-only", sb.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (sbsa_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(sb.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n)
+    assert set(sb.SYMBOLS) <= set(declared_functions())
+
+
+def test_params_struct_layout_matches_c(sb):
+    src = r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "sbsa.h"
+#define F(m) printf("%s %zu\n", #m, offsetof(sbsa_params, m));
+int main(void) {
+  printf("size %zu\n", sizeof(sbsa_params));
+  F(n_q_heads) F(n_kv_heads) F(seq_len) F(head_dim) F(block_size) F(dtype) F(select_mode)
+  F(group_shared) F(index_dim) F(top_k) F(mass_threshold) F(rescue) F(rescue_tau) F(gate)
+  F(gate_margin) F(max_blocks) F(sm_scale) F(score_scale)
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    got = dict(line.split() for line in out.strip().splitlines())
+    assert int(got.pop("size")) == ctypes.sizeof(sb.Params)
+    for name, off in got.items():
+        assert getattr(sb.Params, name).offset == int(off), name
+
+
+def test_status_strings(sb):
+    for code in range(7):
+        assert sb.status_string(code)
+    assert sb.lib.sbsa_version() >= 100
+
+
+def _valid(sb, **kw):
+    base = dict(n_q_heads=4, n_kv_heads=2, seq_len=1000, head_dim=128, block_size=128,
+                dtype="bf16", select_mode="topk", top_k=4)
+    base.update(kw)
+    return sb.make_params(**base)
+
+
+FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced on the host
+
+
+def _select(sb, p):
+    return sb.lib.sbsa_select(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, None)
+
+
+def _attend(sb, p):
+    return sb.lib.sbsa_attend(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None)
+
+
+@pytest.mark.parametrize("mutate,code", [
+    (dict(n_q_heads=3), 1),                      # Hq % Hkv != 0
+    (dict(seq_len=0), 1),
+    (dict(head_dim=96), 2),
+    (dict(block_size=32), 2),
+    (dict(index_dim=32), 2),
+    (dict(top_k=0), 1),
+    (dict(select_mode="cummass", mass_threshold=0.0), 1),
+    (dict(select_mode="cummass", mass_threshold=1.5), 1),
+    (dict(select_mode="cummass", mass_threshold=0.9, gate_margin=0.05), 1),
+    (dict(gate_margin=-1.0), 1),
+    (dict(max_blocks=4), 1),                     # needs k+1 = 5
+    (dict(top_k=4, gate_margin=0.05, max_blocks=5), 1),   # gated needs 2k+1 = 9
+    (dict(select_mode="cummass", mass_threshold=0.9, max_blocks=5), 1),  # needs NB
+    (dict(sm_scale=-1.0), 1),
+])
+def test_invalid_parameters_are_rejected_before_launch(sb, mutate, code):
+    p = _valid(sb, **mutate)
+    assert _select(sb, p) == code
+    assert _attend(sb, p) == code
+    assert sb.lib.sbsa_prefill_workspace_bytes(ctypes.byref(p)) == 0
+
+
+def test_null_pointers_are_rejected(sb):
+    p = _valid(sb)
+    assert sb.lib.sbsa_select(None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == 1
+    assert sb.lib.sbsa_select(ctypes.byref(p), None, FAKE, None, FAKE, FAKE, None, None) == 1
+    assert sb.lib.sbsa_attend(ctypes.byref(p), FAKE, None, FAKE, FAKE, FAKE, FAKE, None) == 1
+    pr = _valid(sb, rescue_tau=1.0)
+    assert sb.lib.sbsa_select(ctypes.byref(pr), FAKE, FAKE, None, FAKE, FAKE, None, None) == 1
+    assert sb.lib.sbsa_pool_blocks(ctypes.byref(p), None, 2, 128, 1, FAKE, None, None) == 1
+
+
+def test_misaligned_pointers_are_rejected(sb):
+    p = _valid(sb)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert sb.lib.sbsa_attend(ctypes.byref(p), odd, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert sb.lib.sbsa_pool_blocks(ctypes.byref(p), odd, 2, 128, 1, FAKE, None, None) == 1
+
+
+def test_pool_argument_checks(sb):
+    p = _valid(sb)
+    assert sb.lib.sbsa_pool_blocks(ctypes.byref(p), FAKE, 3, 128, 2, FAKE, None, None) == 1
+    assert sb.lib.sbsa_pool_blocks(ctypes.byref(p), FAKE, 4, 96, 1, FAKE, None, None) == 2
+    assert sb.lib.sbsa_pool_blocks(ctypes.byref(p), FAKE, 4, 128, 2, FAKE, FAKE, None) == 1
+
+
+def test_fp32_attention_is_limited_to_d64_b64(sb):
+    p = _valid(sb, dtype="fp32")
+    assert _attend(sb, p) == 2
+
+
+def test_workspace_size_and_checks(sb):
+    p = _valid(sb, rescue_tau=5.0)
+    nb = p.n_blocks
+    ws = sb.workspace_bytes(p)
+
+    def r256(x):
+        return (x + 255) // 256 * 256
+    want = (r256(4 * nb * 128 * 4) + r256(2 * nb * 128 * 4) + r256(2 * nb * 4)
+            + r256(4 * nb * p.max_blocks * 4) + r256(4 * nb * 4) + r256(4 * nb))
+    assert ws == want
+    small = sb.lib.sbsa_prefill(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
+                                ws - 1, None, None, None, None)
+    assert small == 3
+    unaligned = sb.lib.sbsa_prefill(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, FAKE,
+                                    ctypes.c_void_p((1 << 20) + 16), ws, None, None, None, None)
+    assert unaligned == 3
+    # index tensors are required when index_dim is set
+    pi = _valid(sb, index_dim=64)
+    assert sb.lib.sbsa_prefill(ctypes.byref(pi), FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
+                               1 << 30, None, None, None, None) == 1

@@ -1,0 +1,307 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle, through
+the C ABI, on the seeded workloads (reduced shapes in full, full shapes on
+sampled query blocks) and on edge cases."""
+import functools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import parity as PT
+from block_sparse_attention_sbsa_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+SMALL_NAMES = ["tiny", "gqa_small", "rbs_small", "gate_small", "msa_small"]
+
+
+@pytest.fixture(scope="module")
+def sb(cuda):
+    from block_sparse_attention_sbsa_b200 import build
+    build.build()
+    from block_sparse_attention_sbsa_b200 import sbsa
+    return sbsa
+
+
+def _oracle_prefill(w, data, **kw):
+    return O.prefill(data["q"], data["k"], data["v"], block=w.block_size, mode=w.select_mode,
+                     top_k_=w.top_k, mass=w.mass_threshold, margin=w.gate_margin,
+                     tau=w.rescue_tau, group_shared=w.group_shared, q_idx=data["q_idx"],
+                     k_idx=data["k_idx"], max_blocks=w.max_blocks, **kw)
+
+
+@functools.lru_cache(maxsize=None)
+def small_case(name):
+    w = W.SMALL[name]
+    data = W.generate(w, "cpu")
+    return w, data, _oracle_prefill(w, data)
+
+
+def _dev(data):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in data.items()}
+
+
+def _kv_of_sel(w):
+    return (lambda hs: hs) if w.group_shared else (lambda hs: hs // w.group)
+
+
+def _all_rows(w):
+    return [(h, i) for h in range(w.n_sel_heads) for i in range(w.n_blocks)]
+
+
+@pytest.mark.parametrize("name", SMALL_NAMES)
+def test_pool_matches_oracle(sb, name):
+    w, data, ref = small_case(name)
+    p = sb.params_for(w)
+    d = _dev(data)
+    ks = d["k_idx"] if w.index_dim else d["k"]
+    qs = d["q_idx"] if w.index_dim else d["q"]
+    c, r = sb.pool_blocks(p, ks, group=1, radius=True)
+    qb, _ = sb.pool_blocks(p, qs, group=w.group if w.group_shared else 1)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(c.cpu().numpy(), ref["c"], rtol=1e-5, atol=2e-5)
+    np.testing.assert_allclose(qb.cpu().numpy(), ref["qbar"], rtol=1e-5, atol=2e-5)
+    if w.rescue_tau is not None:
+        np.testing.assert_allclose(r.cpu().numpy(), ref["r"], rtol=1e-5, atol=2e-5)
+    assert sb.get_status() == sb.OK
+
+
+@pytest.mark.parametrize("name", SMALL_NAMES)
+def test_select_on_oracle_tables(sb, name):
+    """Selection alone: the oracle's pooled tables in, lists out."""
+    w, data, ref = small_case(name)
+    p = sb.params_for(w)
+    qc = torch.tensor(ref["qbar"], dtype=torch.float32, device="cuda")
+    kc = torch.tensor(ref["c"], dtype=torch.float32, device="cuda")
+    kr = torch.tensor(ref["r"], dtype=torch.float32, device="cuda")
+    idx, cnt, flags = sb.select(p, qc, kc, kr if w.rescue_tau is not None else None)
+    idx, cnt, flags = idx.cpu().numpy(), cnt.cpu().numpy(), flags.cpu().numpy()
+    exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
+                                  ref["c"], ref["r"], w, _kv_of_sel(w))
+    assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
+    # padding and flags
+    for hs in range(w.n_sel_heads):
+        for i in range(w.n_blocks):
+            assert np.all(idx[hs, i, cnt[hs, i]:] == -1)
+    same = (idx == ref["idx"]).all(axis=2)
+    assert np.array_equal(flags[same] & 1, ref["flags"][same] & 1)
+    assert sb.get_status() == sb.OK
+
+
+@pytest.mark.parametrize("name", SMALL_NAMES)
+def test_attend_on_oracle_lists(sb, name):
+    """Attention alone, on the oracle's own lists."""
+    w, data, ref = small_case(name)
+    p = sb.params_for(w)
+    d = _dev(data)
+    idx = torch.tensor(ref["idx"], device="cuda")
+    cnt = torch.tensor(ref["cnt"], device="cuda")
+    o = sb.attend(p, d["q"], d["k"], d["v"], idx, cnt)
+    torch.cuda.synchronize()
+    mx, mean = PT.output_errors(o.float().cpu().numpy(), ref["o"])
+    assert sb.get_status() == sb.OK
+    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
+
+
+@pytest.mark.parametrize("name", SMALL_NAMES)
+def test_prefill_end_to_end(sb, name):
+    w, data, ref = small_case(name)
+    p = sb.params_for(w)
+    d = _dev(data)
+    o, idx, cnt, flags = sb.prefill(p, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"])
+    torch.cuda.synchronize()
+    assert sb.get_status() == sb.OK
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
+                                  ref["c"], ref["r"], w, _kv_of_sel(w))
+    assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
+    # outputs on query rows whose lists match the oracle exactly
+    o = o.float().cpu().numpy()
+    same = (idx == ref["idx"]).all(axis=2)
+    mask = np.zeros((w.n_q_heads, w.seq_len), dtype=bool)
+    for h in range(w.n_q_heads):
+        hs = h // w.group if w.group_shared else h
+        for i in range(w.n_blocks):
+            if same[hs, i]:
+                mask[h, i * w.block_size:(i + 1) * w.block_size] = True
+    mx, mean = PT.output_errors(o[mask], ref["o"][mask])
+    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
+
+
+def test_gate_fires_on_the_planted_rows(sb):
+    w, data, ref = small_case("gate_small")
+    p = sb.params_for(w)
+    d = _dev(data)
+    _, idx, cnt, flags = sb.prefill(p, d["q"], d["k"], d["v"])
+    fired = (flags.cpu().numpy() & 1) != 0
+    assert np.array_equal(fired, data["meta"]["tied_rows"].numpy())
+
+
+# ------------------------------------------------------------- full sizes
+
+FULL = ["gqa32k", "rbs128k", "gate64k", "msa512k"]
+
+
+def _sample_blocks(w, meta, count):
+    if w.family == "msa":
+        return W.sample_query_blocks(w, meta, count)
+    g = torch.Generator().manual_seed(w.seed + 11)
+    picks = {w.n_blocks - 1, 0, 1, w.n_blocks // 2}
+    while len(picks) < count:
+        picks.add(int(torch.randint(0, w.n_blocks, (1,), generator=g)))
+    return sorted(picks)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(sb, name):
+    """The benchmark's launch configuration at full size; the oracle checks
+    sampled query blocks (all heads) one by one."""
+    w = W.CONFIGS[name]
+    data = W.generate(w, "cuda")
+    p = sb.params_for(w)
+    call = sb.Prefill(p)
+    o = call(data["q"], data["k"], data["v"], data["q_idx"], data["k_idx"])
+    torch.cuda.synchronize()
+    assert sb.get_status() == sb.OK
+    blocks = _sample_blocks(w, data["meta"], 64 if w.family == "msa" else 24)
+    ks = (data["k_idx"] if w.index_dim else data["k"]).cpu()
+    qs = (data["q_idx"] if w.index_dim else data["q"])
+    c, r = O.pool_keys(ks, w.block_size, with_radius=w.rescue_tau is not None)
+    if r is None:
+        r = np.zeros(c.shape[:2])
+    nb = w.n_blocks
+    qrows = torch.cat([qs[:, i * w.block_size:(i + 1) * w.block_size] for i in blocks], dim=1).cpu()
+    # pooled queries of the sampled blocks only
+    qbar = np.zeros((w.n_sel_heads, nb, w.score_dim))
+    grp = w.group if w.group_shared else 1
+    for bi, i in enumerate(blocks):
+        rows = qrows[:, bi * w.block_size:(bi + 1) * w.block_size]
+        qb = O.pool_queries(rows, w.block_size, group=grp)
+        qbar[:, i] = qb[:, 0]
+    sel_rows = [(hs, i) for hs in range(w.n_sel_heads) for i in blocks]
+    idx, cnt, flags = O.select(qbar, c, r, block_count=nb, mode=w.select_mode, top_k_=w.top_k,
+                               mass=w.mass_threshold, margin=w.gate_margin, tau=w.rescue_tau,
+                               scale=1.0 / math.sqrt(w.score_dim), kv_of_sel=_kv_of_sel(w),
+                               max_blocks=w.max_blocks, rows=sel_rows)
+    gidx = call.idx[:, blocks].cpu().numpy()
+    gcnt = call.cnt[:, blocks].cpu().numpy()
+    gi_full = np.full((w.n_sel_heads, nb, w.max_blocks), -1, dtype=np.int32)
+    gc_full = np.zeros((w.n_sel_heads, nb), dtype=np.int32)
+    gi_full[:, blocks] = gidx
+    gc_full[:, blocks] = gcnt
+    exact, tie = PT.compare_lists(gi_full, gc_full, idx, cnt, sel_rows, qbar, c, r, w,
+                                  _kv_of_sel(w))
+    assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
+    # outputs of the sampled blocks whose lists match (all query heads; two
+    # per group for the 64-head workload); keys/values converted once per
+    # kv head
+    errs = []
+    scale = 1.0 / math.sqrt(w.head_dim)
+    heads_per_group = range(w.group) if w.n_q_heads <= 32 else range(2)
+    for g in range(w.n_kv_heads):
+        kg = data["k"][g].double().cpu().numpy()
+        vg = data["v"][g].double().cpu().numpy()
+        for i in blocks:
+            lo, hi = i * w.block_size, min(w.seq_len, (i + 1) * w.block_size)
+            for hh in heads_per_group:
+                h = g * w.group + hh
+                hs = g if w.group_shared else h
+                if not np.array_equal(gi_full[hs, i], idx[hs, i]):
+                    continue
+                ids = [int(x) for x in idx[hs, i, :cnt[hs, i]]]
+                ref = O.attend_block(data["q"][h, lo:hi].cpu(), kg, vg, ids, i, w.block_size, scale)
+                got = o[h, lo:hi].float().cpu().numpy()
+                errs.append(PT.output_errors(got, ref))
+    assert errs
+    mx = max(e[0] for e in errs)
+    mean = float(np.mean([e[1] for e in errs]))
+    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
+
+
+# ------------------------------------------------------------ edge cases
+
+def _random_case(hq, hk, n, d, b, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    q = torch.randn(hq, n, d, generator=g).to(dt)
+    k = torch.randn(hk, n, d, generator=g).to(dt)
+    v = torch.randn(hk, n, d, generator=g).to(dt)
+    return q, k, v
+
+
+@pytest.mark.parametrize("n,b,d,dtype", [(1, 128, 128, "bf16"), (100, 128, 128, "bf16"),
+                                         (129, 128, 128, "bf16"), (65, 64, 64, "fp32"),
+                                         (700, 64, 128, "bf16"), (300, 128, 64, "bf16"),
+                                         (333, 64, 64, "bf16")])
+def test_ragged_and_tiny_lengths(sb, n, b, d, dtype):
+    q, k, v = _random_case(2, 1, n, d, b, dtype, n + d)
+    nb = O.n_blocks(n, b)
+    p = sb.make_params(n_q_heads=2, n_kv_heads=1, seq_len=n, head_dim=d, block_size=b,
+                       dtype=dtype, top_k=2)
+    o, idx, cnt, _ = sb.prefill(p, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    assert sb.get_status() == sb.OK
+    ref = O.prefill(q, k, v, block=b, mode="topk", top_k_=2, max_blocks=p.max_blocks)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    mx, mean = PT.output_errors(o.float().cpu().numpy(), ref["o"])
+    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
+
+
+def test_all_blocks_kept_is_dense_causal_attention(sb):
+    n, b, d = 1000, 128, 128
+    q, k, v = _random_case(4, 2, n, d, b, "bf16", 5)
+    nb = O.n_blocks(n, b)
+    p = sb.make_params(n_q_heads=4, n_kv_heads=2, seq_len=n, head_dim=d, block_size=b,
+                       top_k=nb)
+    o, idx, cnt, _ = sb.prefill(p, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    dense = torch.nn.functional.scaled_dot_product_attention(
+        q.double().unsqueeze(0), k.double().repeat_interleave(2, 0).unsqueeze(0),
+        v.double().repeat_interleave(2, 0).unsqueeze(0), is_causal=True)[0]
+    mx, mean = PT.output_errors(o.float().cpu().numpy(), dense.numpy())
+    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
+
+
+def test_empty_and_out_of_range_lists(sb):
+    n, b, d = 512, 128, 128
+    q, k, v = _random_case(2, 1, n, d, b, "bf16", 9)
+    nb = O.n_blocks(n, b)
+    p = sb.make_params(n_q_heads=2, n_kv_heads=1, seq_len=n, head_dim=d, block_size=b,
+                       top_k=3, max_blocks=4)
+    idx = np.full((2, nb, 4), -1, dtype=np.int32)
+    cnt = np.zeros((2, nb), dtype=np.int32)
+    # head 0: block 2 lists {0, 3 (future: skipped), 2}; block 3 lists nothing
+    idx[0, 2, :3] = [0, 3, 2]
+    cnt[0, 2] = 3
+    for i in range(nb):
+        idx[1, i, 0] = i
+        cnt[1, i] = 1
+    o = sb.attend(p, q.cuda(), k.cuda(), v.cuda(), torch.tensor(idx, device="cuda"),
+                  torch.tensor(cnt, device="cuda"))
+    st = sb.get_status()
+    assert st == sb.ERR_DEVICE
+    clean = idx.copy()
+    clean[0, 2, :3] = [0, 2, -1]
+    ccnt = cnt.copy()
+    ccnt[0, 2] = 2
+    ref = O.attend(q, k, v, clean, ccnt, block=b, scale=1 / math.sqrt(d), group_shared=False)
+    mx, mean = PT.output_errors(o.float().cpu().numpy(), ref)
+    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
+    assert float(o[0, 3 * b:].abs().max()) == 0.0          # empty list -> zeros
+    assert sb.get_status() == sb.OK                          # cleared on read
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(sb):
+    sb.debug_wait_timeout(2_000_000)                          # 2 ms on a barrier nobody signals
+    assert sb.get_status() == sb.ERR_TIMEOUT
+    assert sb.get_status() == sb.OK
+    w, data, ref = small_case("tiny")
+    d = _dev(data)
+    o, idx, cnt, _ = sb.prefill(sb.params_for(w), d["q"], d["k"], d["v"])
+    torch.cuda.synchronize()
+    assert sb.get_status() == sb.OK
+    mx, _ = PT.output_errors(o.float().cpu().numpy(), ref["o"])
+    assert mx <= PT.MAX_ABS
