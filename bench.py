@@ -49,7 +49,17 @@ def parse_args():
     ap.add_argument("--cpu-blocks", type=int, default=6,
                     help="query blocks (all heads) in the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override the workload length (small cases for profiling)")
     return ap.parse_args()
+
+
+def pick_workload(args):
+    from block_sparse_attention_sbsa_b200 import workloads as W
+    w = W.CONFIGS[args.workload]
+    if args.seq_len:
+        w = w.scaled(name=f"{w.name}@{args.seq_len}", seq_len=args.seq_len)
+    return w
 
 
 def load_peaks():
@@ -204,7 +214,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = W.CONFIGS[args.workload]
+    w = pick_workload(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     data = W.generate(w, dev)
     total_t, total_tok = 0.0, 0
@@ -243,6 +253,27 @@ def workload_config(w):
             "l2": "inputs larger than L2 (Q, K, V each exceed 126 MB); no flush between steps"}
 
 
+# ------------------------------------------------------- rank bookkeeping
+def rank_workload(base, rank: int):
+    """Weak scaling: every rank prefills its own sequence of the same shape."""
+    return base.scaled(seed=base.seed + 1000 * rank)
+
+
+def reduce_max(values, device="cpu"):
+    """Element-wise maximum over ranks (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_throughput(seq_len: int, world: int, steps: int, max_ms: float) -> float:
+    """Tokens of all ranks' sequences over the slowest rank's time."""
+    return seq_len * world * steps / (max_ms / 1000.0)
+
+
 # ------------------------------------------------------------------ GPU arm
 def main():
     args = parse_args()
@@ -261,8 +292,7 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300))
 
-    base = W.CONFIGS[args.workload]
-    w = base.scaled(seed=base.seed + 1000 * rank)   # each rank: its own sequence
+    w = rank_workload(pick_workload(args), rank)
     data = W.generate(w, "cuda")
     p = sbsa.params_for(w)
     st = sbsa.Staged(p)
@@ -352,19 +382,15 @@ def main():
         raise RuntimeError(f"device status after e2e: {sbsa.status_string(stat)}")
 
     # ---- max over ranks ----
-    vals = torch.tensor([elapsed_ms, e2e_ms, att_ms, pool_ms, sel_ms], device="cuda",
-                        dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms, att_ms, pool_ms, sel_ms = [float(x) for x in vals.tolist()]
+    elapsed_ms, e2e_ms, att_ms, pool_ms, sel_ms = reduce_max(
+        [elapsed_ms, e2e_ms, att_ms, pool_ms, sel_ms], device="cuda")
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return 0
 
     peaks, src = load_peaks()
-    tokens = w.seq_len * world * args.steps
-    value = tokens / (elapsed_ms / 1000.0)
+    value = weak_throughput(w.seq_len, world, args.steps, elapsed_ms)
     ms_per_step = elapsed_ms / args.steps
     att_tflops = attend_flops / (att_ms / 1000.0) / 1e12
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -401,7 +427,7 @@ def main():
         "attended_pairs": pairs,
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
-        "e2e": {"value": w.seq_len * world * args.e2e_steps / (e2e_ms / 1000.0), "unit": UNIT,
+        "e2e": {"value": weak_throughput(w.seq_len, world, args.e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "pinned host -> device copies, sbsa_prefill, device -> host copy of O"},
     }

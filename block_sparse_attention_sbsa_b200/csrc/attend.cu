@@ -79,6 +79,11 @@ struct Cfg {
   static constexpr int TM_COLS_ = pow2_at_least(2 * BN + D);
   static constexpr int SMEM_FLOOR = 233472 / (512 / TM_COLS_ + 1) + 1024;
   static constexpr int SMEM_BYTES = SMEM_USED > SMEM_FLOOR ? SMEM_USED : SMEM_FLOOR;
+  // V is read MN-major: 16-bit types use the 128-byte swizzle of 16-byte
+  // chunks (8-row period), 32-bit types the 128-byte swizzle of 32-byte
+  // chunks (4-row period), the only MN-major layout tf32 operands accept.
+  static constexpr uint32_t V_LAYOUT = ES == 4 ? kSwizzle128B_32BAtom : kSwizzle128B;
+  static constexpr uint32_t V_SBO = ES == 4 ? 512 : 1024;
   static constexpr int TM_S = 0;
   static constexpr int TM_O = 2 * BN;
   static constexpr int TM_COLS = pow2_at_least(2 * BN + D);
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         for (int kk = 0; kk < BN / C::KSTEP; ++kk) {
           const int kb = kk * 32;  // byte offset along keys in the P rows
           const uint64_t ad = smem_desc(a0 + (kb / 128) * (BM * 128) + (kb % 128), 16, 1024);
-          const uint64_t bd = smem_desc(b0 + kk * C::KSTEP * 128, BN * 128, 1024);
+          const uint64_t bd = smem_desc(b0 + kk * C::KSTEP * 128, BN * 128, C::V_SBO, C::V_LAYOUT);
           if constexpr (C::ES == 2)
             umma_f16_ss(tmem + C::TM_O, ad, bd, C::IDESC_O, (m > 0 || kk > 0) ? 1u : 0u);
           else
@@ -492,7 +497,7 @@ EncodeTiledFn encode_fn() {
 // 3-D map over a [heads, N, d] tensor: box = one 128-byte row segment of
 // `rows` consecutive tokens of one head, 128-byte swizzle, zero fill outside.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, int heads,
-              int n, int d, int rows) {
+              int n, int d, int rows, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)heads};
@@ -500,7 +505,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* bas
   cuuint32_t box[3] = {(cuuint32_t)(128 / esize), (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -512,7 +517,8 @@ int launch_typed(const AttendArgs& a, cudaStream_t stream) {
   const CUtensorMapDataType dt = Elem<T>::tma;
   if (!make_map(&p.tm_q, dt, C::ES, a.q, a.hq, a.n, D, BM) ||
       !make_map(&p.tm_k, dt, C::ES, a.k, a.hkv, a.n, D, BM) ||
-      !make_map(&p.tm_v, dt, C::ES, a.v, a.hkv, a.n, D, BM))
+      !make_map(&p.tm_v, dt, C::ES, a.v, a.hkv, a.n, D, BM,
+                C::ES == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B))
     return SBSA_ERR_CUDA;
   p.o = a.o;
   p.idx = a.idx;

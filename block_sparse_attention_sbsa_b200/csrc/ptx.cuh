@@ -190,15 +190,20 @@ __device__ __forceinline__ void tmem_wait_st() {
 // Shared-memory matrix descriptor (sm_100): start address >> 4 in bits
 // [0,14), leading byte offset >> 4 in [16,30), stride byte offset >> 4 in
 // [32,46), the fixed version value 1 in [46,48), base offset 0 in [49,52),
-// layout type in [61,64) (2 = 128-byte swizzle).
+// layout type in [61,64): 2 = 128-byte swizzle of 16-byte chunks, 1 =
+// 128-byte swizzle of 32-byte chunks (the MN-major layout of 32-bit operands).
+constexpr uint32_t kSwizzle128B = 2;
+constexpr uint32_t kSwizzle128B_32BAtom = 1;
+
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes,
-                                              uint32_t sbo_bytes) {
+                                              uint32_t sbo_bytes,
+                                              uint32_t layout = kSwizzle128B) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
+  d |= (uint64_t)(layout & 7u) << 61;
   return d;
 }
 

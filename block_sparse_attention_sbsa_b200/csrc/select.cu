@@ -29,7 +29,8 @@ namespace {
 
 constexpr int kSelThreads = 256;
 constexpr int kWarps = kSelThreads / 32;
-constexpr int kJC = 128;  // candidate key blocks per scoring chunk
+constexpr int kJC = 128;      // candidate key blocks per scoring chunk
+constexpr int kMaxWalk = 24;  // ranked-walk steps before the radix fallback
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
@@ -58,6 +59,21 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
   return v;
 }
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t w = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
+
+// Unique descending order of the candidates: score key first, then the lower
+// block id (ids are complemented so that a larger composite ranks first).
+__device__ __forceinline__ uint64_t rank_key(float s, int j) {
+  return ((uint64_t)fkey(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+}
+
 __device__ __forceinline__ uint32_t warp_max_u(uint32_t v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
@@ -154,9 +170,21 @@ __device__ uint32_t radix_select_mass(const float* s, int n, float smax, double 
       const float sv = in ? s[j] : 0.f;
       const uint32_t u = in ? fkey(sv) : 0u;
       const bool match = in && ((u & pmask) == prefix);
+      const uint32_t bin = (u >> shift) & 0xFFu;
+      uint64_t w = match ? mass_weight(sv, smax, wscale) : 0ull;
+      const unsigned act = __ballot_sync(0xFFFFFFFFu, match);
       if (match) {
-        const uint64_t w = mass_weight(sv, smax, wscale);
-        if (w) atomicAdd(&hist[(u >> shift) & 0xFFu], (unsigned long long)w);
+        // lanes sharing a bin add their weights through one atomic
+        const unsigned peers = __match_any_sync(act, bin);
+        const int leader = __ffs(peers) - 1;
+        unsigned rest = peers & ~(1u << leader);
+        while (rest) {
+          const int src = __ffs(rest) - 1;
+          rest &= rest - 1;
+          const uint64_t other = __shfl_sync(peers, w, src);
+          if (lane == leader) w += other;
+        }
+        if (lane == leader && w) atomicAdd(&hist[bin], (unsigned long long)w);
       }
     }
     __syncwarp();
@@ -285,6 +313,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
     uint32_t vkey = 0xFFFFFFFFu;
     int take_eq = 0;
     bool select_all = false;
+    bool walked = false;  // cumulative mass decided by the ranked walk
+    uint64_t wkey = 0;    // rank key of the last block the walk kept
     uint8_t flag = 0;
     if (a.mode == SBSA_TOPK) {
       int kk = a.top_k;
@@ -341,25 +371,50 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
         for (int j = lane; j < n; j += 32) z += (double)__expf(s[j] - m);
         z = warp_sum_d(z);
         const double wscale = 1152921504606846976.0 / z;  // 2^60 / Z
-        uint64_t wtot = 0;
-        for (int j = lane; j < n; j += 32) wtot += mass_weight(s[j], m, wscale);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) wtot += __shfl_xor_sync(0xFFFFFFFFu, wtot, o);
-        double tgt_d = ceil((double)a.mass * 1152921504606846976.0);
-        uint64_t target = (uint64_t)tgt_d;
-        if (target > wtot) target = wtot;
-        if (target == 0) target = 1;
-        if (wtot == 0) {
-          select_all = true;
+        const uint64_t want = (uint64_t)ceil((double)a.mass * 1152921504606846976.0);
+        // The kept prefix is usually a handful of blocks: walk the ranked
+        // order one maximum at a time, accumulating fixed-point mass in the
+        // same order as the definition (descending score, lower id first).
+        uint64_t prev = ~0ull, cum = 0;
+        int taken = 0;
+        for (; taken < kMaxWalk && taken < n; ++taken) {
+          uint64_t best = 0;
+          for (int j = lane; j < n; j += 32) {
+            const uint64_t c = rank_key(s[j], j);
+            if (c < prev && c > best) best = c;
+          }
+          best = warp_max_u64(best);
+          prev = best;
+          cum += mass_weight(key_float((uint32_t)(best >> 32)), m, wscale);
+          if (cum >= want) {
+            walked = true;
+            break;
+          }
+        }
+        if (walked) {
+          wkey = prev;
+        } else if (taken == n) {
+          select_all = true;  // rounding kept the total below the threshold
         } else {
-          uint64_t w_gt;
-          vkey = radix_select_mass(s, n, m, wscale, target, hist64, &w_gt);
-          const uint64_t w_one = mass_weight(key_float(vkey), m, wscale);
-          // tied keys all carry w_one; take the fewest that reach the target
-          uint64_t t = w_one ? (target - w_gt + w_one - 1) / w_one : 1;
-          if (t < 1) t = 1;
-          if (t > (uint64_t)n) t = (uint64_t)n;
-          take_eq = (int)t;
+          // long prefix: exact radix selection on mass histograms
+          uint64_t wtot = 0;
+          for (int j = lane; j < n; j += 32) wtot += mass_weight(s[j], m, wscale);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) wtot += __shfl_xor_sync(0xFFFFFFFFu, wtot, o);
+          uint64_t target = want > wtot ? wtot : want;
+          if (target == 0) target = 1;
+          if (wtot == 0) {
+            select_all = true;
+          } else {
+            uint64_t w_gt;
+            vkey = radix_select_mass(s, n, m, wscale, target, hist64, &w_gt);
+            const uint64_t w_one = mass_weight(key_float(vkey), m, wscale);
+            // tied keys all carry w_one; take the fewest that reach the target
+            uint64_t t = w_one ? (target - w_gt + w_one - 1) / w_one : 1;
+            if (t < 1) t = 1;
+            if (t > (uint64_t)n) t = (uint64_t)n;
+            take_eq = (int)t;
+          }
         }
       }
     }
@@ -386,6 +441,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
       if (in) {
         if (select_all) {
           basesel = true;
+        } else if (walked) {
+          basesel = rank_key(s[j], j) >= wkey;
         } else {
           const uint32_t u = fkey(s[j]);
           basesel = u > vkey;
