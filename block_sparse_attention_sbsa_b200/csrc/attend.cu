@@ -23,10 +23,12 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include <mutex>
+#include <cstdlib>
+#include <cstring>
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "tma_map.h"
 
 namespace sbsa {
 namespace {
@@ -474,42 +476,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
   }
 }
 
-// ------------------------------------------------------------------ host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  });
-  return fn;
-}
-
-// 3-D map over a [heads, N, d] tensor: box = one 128-byte row segment of
-// `rows` consecutive tokens of one head, 128-byte swizzle, zero fill outside.
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, int heads,
-              int n, int d, int rows, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)d * esize, (cuuint64_t)n * d * esize};
-  cuuint32_t box[3] = {(cuuint32_t)(128 / esize), (cuuint32_t)rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <typename T, int BM, int D>
 int launch_typed(const AttendArgs& a, cudaStream_t stream) {
   using C = Cfg<T, BM, D>;
@@ -565,6 +531,16 @@ cudaError_t launch_wait_probe(uint64_t timeout_ns, int* status, cudaStream_t str
 }
 
 int launch_attend(const AttendArgs& a, cudaStream_t stream) {
+  static const bool single = [] {
+    const char* e = std::getenv("SBSA_ATTEND_KERNEL");
+    return e && std::strcmp(e, "single") == 0;
+  }();
+  if (!single && a.dtype == SBSA_BF16 && a.block == 128 && (a.d == 128 || a.d == 64))
+    return launch_attend_pingpong(a, stream);
+  return launch_attend_single(a, stream);
+}
+
+int launch_attend_single(const AttendArgs& a, cudaStream_t stream) {
   if (a.dtype == SBSA_BF16) {
     if (a.block == 128 && a.d == 128) return launch_typed<__nv_bfloat16, 128, 128>(a, stream);
     if (a.block == 128 && a.d == 64) return launch_typed<__nv_bfloat16, 128, 64>(a, stream);

@@ -305,3 +305,31 @@ def test_bounded_wait_reports_timeout_and_context_survives(sb):
     assert sb.get_status() == sb.OK
     mx, _ = PT.output_errors(o.float().cpu().numpy(), ref["o"])
     assert mx <= PT.MAX_ABS
+
+
+def test_single_tile_kernel_matches_oracle_too(sb):
+    """The one-tile-per-CTA attention kernel (selected by SBSA_ATTEND_KERNEL)
+    on the 128-token-block workloads, in a child process."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, 'tests'); sys.path.insert(0, '.');\n"
+        "import test_gpu_parity as T, numpy as np, torch\n"
+        "from block_sparse_attention_sbsa_b200 import sbsa\n"
+        "import parity as PT\n"
+        "for name in ['gqa_small', 'rbs_small', 'msa_small']:\n"
+        "    w, data, ref = T.small_case(name)\n"
+        "    d = T._dev(data)\n"
+        "    o = sbsa.attend(sbsa.params_for(w), d['q'], d['k'], d['v'],\n"
+        "                    torch.tensor(ref['idx'], device='cuda'), torch.tensor(ref['cnt'], device='cuda'))\n"
+        "    torch.cuda.synchronize()\n"
+        "    assert sbsa.get_status() == sbsa.OK\n"
+        "    mx, mean = PT.output_errors(o.float().cpu().numpy(), ref['o'])\n"
+        "    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (name, mx, mean)\n"
+        "print('single ok')\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SBSA_ATTEND_KERNEL="single")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0 and "single ok" in r.stdout, r.stdout + r.stderr
