@@ -536,7 +536,7 @@ int launch_attend(const AttendArgs& a, cudaStream_t stream) {
     return e && std::strcmp(e, "single") == 0;
   }();
   if (!single && a.dtype == SBSA_BF16 && a.block == 128 && (a.d == 128 || a.d == 64))
-    return launch_attend_pingpong(a, stream);
+    return launch_attend_persistent(a, stream);
   return launch_attend_single(a, stream);
 }
 

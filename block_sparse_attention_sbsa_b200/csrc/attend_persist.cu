@@ -1,0 +1,538 @@
+// Attention over the selected key blocks: persistent, deeply pipelined
+// version for bf16 with 128-token blocks (the long-context workloads).
+//
+// "RBS-Attention" (iaonda.com), method paragraph: sparse prefill compatible
+// with sparse FlashAttention, i.e. exact softmax attention restricted to the
+// kept blocks.  "MiniMax presenta MSA", "Que es MSA y como funciona?": full
+// attention over the preselected blocks only.
+//
+// One CTA per SM walks a static list of (query head, query block) items,
+// longest lists first.  The listed key blocks of consecutive items form one
+// stream indexed by a CTA-wide block counter g, so loads and products run
+// ahead across item boundaries.  10 warps:
+//   warp 0     TMA producer: Q of item t into Q[t % 2]; K_j, V_j of block g
+//              into a 4-stage ring (positions 2g, 2g + 1).
+//   warp 1     TMEM owner and single-thread MMA issuer, in the order
+//              S(0), S(1), PV(0), S(2), PV(1), ...:
+//                S(g)  = Q K_j^T        -> TMEM S[g % 2]
+//                PV(g) : O[t % 2] += P(g) V_j, with P(g) (bf16) read from the
+//                        first half of S[g % 2], where the softmax wrote it.
+//   warps 2-5  softmax: one query row per thread; S row -> running maximum
+//              (moved, and O rescaled in TMEM, only when it grows by more
+//              than 2^8) -> P; row sums handed to the epilogue per item.
+//   warps 6-9  epilogue: O[t % 2] / l -> global memory, overlapping the next
+//              item's products.
+// Every wait is bounded (2 s); on expiry the CTA records SBSA_ERR_TIMEOUT,
+// stops issuing, drains its copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tma_map.h"
+
+namespace sbsa {
+namespace {
+
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D>
+struct PS {
+  static constexpr int BM = 128;
+  static constexpr int BN = 128;
+  static constexpr int NA_D = D / 64;  // 128-byte swizzle atoms across d (bf16)
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;                            // Q[2]
+  static constexpr int OFF_KV = 2 * Q_BYTES;                 // ring[kStages]
+  static constexpr int OFF_L = OFF_KV + kStages * KV_BYTES;  // row sums [2][BM]
+  static constexpr int OFF_BAR = OFF_L + 2 * BM * 4;
+  // q_full[2] q_free[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done[2]
+  // o_full[2] o_free[2] l_full[2] drain
+  static constexpr int NBARS = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int TM_S = 0;       // S[0], S[1]: 2 x BN columns
+  static constexpr int TM_O = 2 * BN;  // O[0], O[1]: 2 x D columns
+  static constexpr int TM_COLS = 512;
+  static constexpr uint32_t IDESC_S = make_idesc(1, BM, BN, false, false);
+  static constexpr uint32_t IDESC_O = make_idesc(1, BM, D, false, true);
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(2 * BN + 2 * D <= TM_COLS, "TMEM budget");
+};
+
+struct PSParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  void* o;
+  const int32_t* idx;
+  const int32_t* cnt;
+  int hq, n, nb, group, group_shared, kmax, total;
+  float scale_log2;
+  int* status;
+};
+
+struct Item {
+  int i, h, g, count, valid;
+  const int32_t* list;
+};
+
+// Item number t of this CTA (static round robin over the longest-first
+// order); `valid` counts the list entries inside [0, i].
+__device__ __forceinline__ bool load_item(const PSParams& p, int t, Item& it) {
+  const long long item = (long long)blockIdx.x + (long long)t * gridDim.x;
+  if (item >= p.total) return false;
+  it.i = p.nb - 1 - (int)(item / p.hq);
+  it.h = (int)(item % p.hq);
+  it.g = it.h / p.group;
+  const int hs = p.group_shared ? it.g : it.h;
+  it.list = p.idx + ((size_t)hs * p.nb + it.i) * p.kmax;
+  const int c = p.cnt[(size_t)hs * p.nb + it.i];
+  it.count = c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
+  int v = 0;
+  for (int r = 0; r < it.count; ++r) {
+    const int j = it.list[r];
+    v += (j >= 0 && j <= it.i) ? 1 : 0;
+  }
+  it.valid = v;
+  return true;
+}
+
+__device__ __forceinline__ bool valid_entry(const Item& it, int j) { return j >= 0 && j <= it.i; }
+
+__device__ __forceinline__ void record(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_constant__ PSParams p) {
+  using C = PS<D>;
+  constexpr int BM = C::BM, BN = C::BN;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  unsigned char* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bar;
+  uint64_t* q_free = q_full + 2;
+  uint64_t* kv_full = q_free + 2;
+  uint64_t* kv_empty = kv_full + kStages;
+  uint64_t* s_full = kv_empty + kStages;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* o_full = pv_done + 2;
+  uint64_t* o_free = o_full + 2;
+  uint64_t* l_full = o_free + 2;
+  uint64_t* drain = l_full + 2;
+  float* l_buf = reinterpret_cast<float*>(smem + C::OFF_L);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  unsigned char* sQ = smem + C::OFF_Q;
+  unsigned char* sKV = smem + C::OFF_KV;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_free[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_free[b], 128);
+      mbar_init(&l_full[b], 128);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&](int code) {
+    *abort_flag = 1;
+    record(p.status, code);
+  };
+  auto wait = [&](uint64_t* b, uint32_t parity) {
+    return mbar_wait_bounded(b, parity, abort_flag, kTimeoutNs);
+  };
+
+  if (warp == 0) {
+    // ================================================================ TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      int pos = 0, t = 0, q_loaded = 0;
+      bool ok = true;
+      Item it;
+      for (; ok && load_item(p, t, it); ++t) {
+        const int qb = t & 1;
+        if (t >= 2 && !wait(&q_free[qb], ((t - 2) >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
+        for (int a = 0; a < C::NA_D; ++a)
+          tma_load_3d(sQ + qb * C::Q_BYTES + a * (BM * 128), &p.tm_q, &q_full[qb], a * 64,
+                      it.i * BM, it.h);
+        q_loaded = t + 1;
+        for (int r = 0; ok && r < it.count; ++r) {
+          const int j = it.list[r];
+          if (!valid_entry(it, j)) {
+            record(p.status, SBSA_ERR_DEVICE);
+            continue;
+          }
+          for (int half = 0; half < 2; ++half) {
+            const int st = pos % kStages;
+            if (!wait(&kv_empty[st], ((pos / kStages) & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
+            const CUtensorMap* m = half ? &p.tm_v : &p.tm_k;
+            for (int a = 0; a < C::NA_D; ++a)
+              tma_load_3d(sKV + st * C::KV_BYTES + a * (BN * 128), m, &kv_full[st], a * 64,
+                          j * BN, it.g);
+            ++pos;
+          }
+        }
+      }
+      volatile int never = 0;
+      const int first = pos > kStages ? pos - kStages : 0;
+      if (!ok) {
+        if (!*abort_flag) fail(SBSA_ERR_TIMEOUT);
+        // drain copies still landing in shared memory
+        for (int u = (q_loaded >= 2 ? q_loaded - 2 : 0); u < q_loaded; ++u)
+          mbar_wait_bounded(&q_full[u & 1], (u >> 1) & 1, &never, kTimeoutNs);
+        for (int q = first; q < pos; ++q)
+          mbar_wait_bounded(&kv_full[q % kStages], (q / kStages) & 1, &never, kTimeoutNs);
+      } else {
+        // wait for the MMA thread's last asynchronous releases
+        for (int q = first; q < pos; ++q)
+          if (!wait(&kv_empty[q % kStages], (q / kStages) & 1)) break;
+        for (int u = (q_loaded >= 2 ? q_loaded - 2 : 0); u < q_loaded; ++u)
+          if (!wait(&q_free[u & 1], (u >> 1) & 1)) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t kv_base = smem_u32(sKV);
+      struct Pending {
+        int g, t, b, last;  // block counter, item, block within item, last of item
+      };
+      Pending prev{0, 0, 0, 0};
+      bool have_prev = false, ok = true;
+      auto issue_pv = [&](const Pending& pv) -> bool {
+        if (!wait(&p_full[pv.g & 1], (pv.g >> 1) & 1)) return false;
+        if (pv.b == 0 && pv.t >= 2 && !wait(&o_free[pv.t & 1], ((pv.t - 2) >> 1) & 1))
+          return false;
+        const int vpos = 2 * pv.g + 1;
+        const int st = vpos % kStages;
+        if (!wait(&kv_full[st], (vpos / kStages) & 1)) return false;
+        tc_fence_after();
+        const uint32_t v_base = kv_base + st * C::KV_BYTES;
+        const uint32_t a_col = tmem + C::TM_S + (pv.g & 1) * BN;
+        const uint32_t o_col = tmem + C::TM_O + (pv.t & 1) * D;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bd = smem_desc(v_base + kk * 16 * 128, BN * 128, 1024);
+          umma_f16_ts(o_col, a_col + kk * 8, bd, C::IDESC_O, (pv.b > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&kv_empty[st]);
+        umma_commit(&pv_done[pv.g & 1]);
+        if (pv.last) umma_commit(&o_full[pv.t & 1]);
+        return true;
+      };
+      int g = 0, t = 0;
+      Item it;
+      for (; ok && load_item(p, t, it); ++t) {
+        const int qb = t & 1;
+        if (!wait(&q_full[qb], (t >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (it.valid == 0) {
+          // nothing to multiply: release Q; the epilogue writes zeros
+          umma_commit(&q_free[qb]);
+          umma_commit(&o_full[qb]);
+          continue;
+        }
+        int b = 0;
+        for (int r = 0; r < it.count; ++r) {
+          const int j = it.list[r];
+          if (!valid_entry(it, j)) continue;
+          const int kpos = 2 * g;
+          const int st = kpos % kStages;
+          if (!wait(&kv_full[st], (kpos / kStages) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qa = q_base + qb * C::Q_BYTES;
+          const uint32_t ka = kv_base + st * C::KV_BYTES;
+          const uint32_t s_col = tmem + C::TM_S + (g & 1) * BN;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int kb = kk * 32;
+            const uint64_t ad = smem_desc(qa + (kb / 128) * (BM * 128) + (kb % 128), 16, 1024);
+            const uint64_t bd = smem_desc(ka + (kb / 128) * (BN * 128) + (kb % 128), 16, 1024);
+            umma_f16_ss(s_col, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&kv_empty[st]);
+          umma_commit(&s_full[g & 1]);
+          const bool last = (b == it.valid - 1);
+          if (last) umma_commit(&q_free[qb]);
+          if (have_prev && !issue_pv(prev)) {
+            ok = false;
+            break;
+          }
+          prev = Pending{g, t, b, last ? 1 : 0};
+          have_prev = true;
+          ++g;
+          ++b;
+        }
+      }
+      if (ok && have_prev) ok = issue_pv(prev);
+      if (!ok) {
+        if (!*abort_flag) fail(SBSA_ERR_TIMEOUT);
+        umma_commit(drain);
+        volatile int never = 0;
+        mbar_wait_bounded(drain, 0, &never, kTimeoutNs);
+      }
+    }
+  } else if (warp < 6) {
+    // ================================================================ softmax
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    int g = 0;
+    bool ok = true;
+    Item it;
+    for (int t = 0; ok && load_item(p, t, it); ++t) {
+      float m_run = -INFINITY, l_run = 0.f;
+      const uint32_t o_col = tmem + lane_base + C::TM_O + (t & 1) * D;
+      int b = 0;
+      for (int r = 0; r < it.count; ++r) {
+        const int j = it.list[r];
+        if (!valid_entry(it, j)) continue;
+        const bool diag = (j == it.i);
+        const uint32_t s_col = tmem + lane_base + C::TM_S + (g & 1) * BN;
+        if (!wait(&s_full[g & 1], (g >> 1) & 1)) ok = false;
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // pass 1: row maximum (64 columns at a time)
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 64) {
+          float a[32], bb[32];
+          tmem_ld32(s_col + c0, a);
+          tmem_ld32(s_col + c0 + 32, bb);
+          tmem_wait_ld();
+          if (diag) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (c0 + c <= row) mx = fmaxf(mx, a[c]);
+              if (c0 + 32 + c <= row) mx = fmaxf(mx, bb[c]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(a[c], bb[c]));
+          }
+        }
+        const float m_new = fmaxf(m_run, mx * p.scale_log2);
+        if (b == 0) {
+          m_run = m_new;
+        } else if (__any_sync(0xFFFFFFFFu, m_new > m_run + kRescaleLog2)) {
+          // O must hold PV(g - 1) before it is rescaled
+          if (!wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) ok = false;
+          if (!__all_sync(0xFFFFFFFFu, ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float alpha = ex2_approx(m_run - m_new);
+          l_run *= alpha;
+          m_run = m_new;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float o[32];
+            tmem_ld32(o_col + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] *= alpha;
+            tmem_st32(o_col + c0, o);
+          }
+        }
+        // pass 2: P = exp2(S * scale - m) as bf16 over the first half of the
+        // S columns (step c0 reads S[c0, c0+64), writes P to [c0/2, c0/2+32),
+        // columns whose S values were already read)
+        float lsum = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 64) {
+          float a[32], bb[32];
+          tmem_ld32(s_col + c0, a);
+          tmem_ld32(s_col + c0 + 32, bb);
+          tmem_wait_ld();
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
+            float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
+            float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
+            float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
+            if (diag) {
+              if (c0 + c > row) p0 = 0.f;
+              if (c0 + c + 1 > row) p1 = 0.f;
+              if (c0 + 32 + c > row) p2 = 0.f;
+              if (c0 + 32 + c + 1 > row) p3 = 0.f;
+            }
+            lsum += (p0 + p1) + (p2 + p3);
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+            pk[16 + (c >> 1)] = pack_bf16x2(p2, p3);
+          }
+          tmem_st32u(s_col + (c0 >> 1), pk);
+        }
+        l_run += lsum;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[g & 1]);
+        ++g;
+        ++b;
+      }
+      if (!ok) break;
+      // hand the row sum to the epilogue once it is done with item t - 2
+      if (t >= 2 && !wait(&o_free[t & 1], ((t - 2) >> 1) & 1)) ok = false;
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        ok = false;
+        break;
+      }
+      l_buf[(t & 1) * BM + row] = (b > 0) ? l_run : 0.f;
+      mbar_arrive(&l_full[t & 1]);
+    }
+    if (!ok && lane == 0 && !*abort_flag) fail(SBSA_ERR_TIMEOUT);
+  } else {
+    // ================================================================ epilogue
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    bool ok = true;
+    Item it;
+    for (int t = 0; ok && load_item(p, t, it); ++t) {
+      if (!wait(&l_full[t & 1], (t >> 1) & 1)) ok = false;
+      if (ok && !wait(&o_full[t & 1], (t >> 1) & 1)) ok = false;
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float l = l_buf[(t & 1) * BM + row];
+      const float inv_l = (it.valid > 0 && l > 0.f) ? 1.f / l : 0.f;
+      const int tok = it.i * BM + row;
+      const bool store = tok < p.n;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + ((size_t)it.h * p.n + tok) * D;
+      const uint32_t o_col = tmem + lane_base + C::TM_O + (t & 1) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float o[32];
+        if (it.valid > 0) {
+          tmem_ld32(o_col + c0, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0.f;
+        }
+        if (store) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(o[c + 0] * inv_l, o[c + 1] * inv_l);
+            v.y = pack_bf16x2(o[c + 2] * inv_l, o[c + 3] * inv_l);
+            v.z = pack_bf16x2(o[c + 4] * inv_l, o[c + 5] * inv_l);
+            v.w = pack_bf16x2(o[c + 6] * inv_l, o[c + 7] * inv_l);
+            *reinterpret_cast<uint4*>(orow + c0 + c) = v;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&o_free[t & 1]);
+    }
+    if (!ok && lane == 0 && !*abort_flag) fail(SBSA_ERR_TIMEOUT);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+template <int D>
+int launch_d(const AttendArgs& a, cudaStream_t stream) {
+  using C = PS<D>;
+  PSParams p{};
+  const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&p.tm_q, dt, 2, a.q, a.hq, a.n, D, 128) ||
+      !make_map(&p.tm_k, dt, 2, a.k, a.hkv, a.n, D, 128) ||
+      !make_map(&p.tm_v, dt, 2, a.v, a.hkv, a.n, D, 128))
+    return SBSA_ERR_CUDA;
+  p.o = a.o;
+  p.idx = a.idx;
+  p.cnt = a.cnt;
+  p.hq = a.hq;
+  p.n = a.n;
+  p.nb = (a.n + 127) / 128;
+  p.group = a.hq / a.hkv;
+  p.group_shared = a.group_shared;
+  p.kmax = a.kmax;
+  p.total = a.hq * p.nb;
+  p.scale_log2 = a.sm_scale * 1.4426950408889634f;
+  p.status = a.status;
+  auto kern = attend_ps_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return SBSA_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return SBSA_ERR_CUDA;
+  const int grid = p.total < sms ? p.total : sms;
+  kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SBSA_OK : SBSA_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_attend_persistent(const AttendArgs& a, cudaStream_t stream) {
+  if (a.dtype != SBSA_BF16 || a.block != 128) return SBSA_ERR_UNSUPPORTED;
+  if (a.d == 128) return launch_d<128>(a, stream);
+  if (a.d == 64) return launch_d<64>(a, stream);
+  return SBSA_ERR_UNSUPPORTED;
+}
+
+}  // namespace sbsa

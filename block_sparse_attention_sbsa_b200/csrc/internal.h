@@ -59,7 +59,7 @@ struct AttendArgs {
 };
 
 // Returns an SBSA_* code (SBSA_ERR_CUDA on launch/driver failure).  bf16
-// with 128-token blocks runs the persistent two-tile kernel unless the
+// with 128-token blocks runs the persistent pipelined kernel unless the
 // environment variable SBSA_ATTEND_KERNEL is "single"; every other
 // combination runs the one-tile-per-CTA kernel.
 int launch_attend(const AttendArgs& a, cudaStream_t stream);
@@ -67,8 +67,8 @@ int launch_attend(const AttendArgs& a, cudaStream_t stream);
 // The one-tile-per-CTA kernel (every supported dtype / block / d).
 int launch_attend_single(const AttendArgs& a, cudaStream_t stream);
 
-// The persistent two-tile kernel (bf16, B = 128, d in {64, 128}).
-int launch_attend_pingpong(const AttendArgs& a, cudaStream_t stream);
+// The persistent pipelined kernel (bf16, B = 128, d in {64, 128}).
+int launch_attend_persistent(const AttendArgs& a, cudaStream_t stream);
 
 // One CTA waiting on an mbarrier that never completes, through the bounded
 // wait of the pipelines; records SBSA_ERR_TIMEOUT when the limit expires.
