@@ -414,7 +414,7 @@ def main():
             "bound": "tensor", "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",
             "frac": att_tflops / peak_tf,
             "traffic": NCU_ATTEND_TRAFFIC.get(w.name),
-            "kernel": "attend_kernel (tcgen05, bf16, B=128, d=128)",
+            "kernel": "attend_ps_kernel<128> (persistent, tcgen05, bf16, B=128, d=128)",
             "note": f"peak = bf16_tflops burst, of {src}; achieved = 4*d*unmasked pairs / mean launch time",
         },
         "selection_roofline": {

@@ -3,7 +3,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
-#include "../../include/sbsa.h"
+#include "sbsa.h"
 
 namespace sbsa {
 
