@@ -173,6 +173,41 @@ int sbsa_version(void);
  */
 int sbsa_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
+/*
+ * sbsa_prefill_noalloc -- sbsa_prefill for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is a deployment
+ * convenience of this library.
+ *
+ * Some callers have no way to supply a workspace: a plugin inside a host
+ * framework that owns all device memory and gives its operators no
+ * allocator, a latency-critical path where cudaMalloc's implicit device
+ * synchronisation is not acceptable, or a process whose device memory
+ * budget is fixed at start-up.  This entry point takes the same inputs and
+ * outputs as sbsa_prefill minus the workspace; its temporaries (pooled
+ * tables and, when idx_out/cnt_out are NULL, the block lists) live in one
+ * fixed array of SBSA_NOALLOC_SCRATCH_BYTES compiled into the library.  It
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *  - Limit: problems whose temporaries exceed SBSA_NOALLOC_SCRATCH_BYTES are
+ *    rejected with SBSA_ERR_WORKSPACE before anything is launched (pass
+ *    idx_out/cnt_out to keep the lists out of the scratch).
+ *  - Memory: every GPU that loads the library holds the array (32 MiB) until
+ *    the process exits.
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Sharing: all calls on a device use the same array and it keeps the last
+ *    call's contents.  Nothing in it needs to start at zero (every byte a
+ *    call reads is written earlier by the same call), but calls whose kernels
+ *    overlap on the GPU (different streams without ordering) race on it:
+ *    serialise them.
+ * Arguments, layouts and errors otherwise as sbsa_prefill.
+ */
+#define SBSA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int sbsa_prefill_noalloc(const sbsa_params* p, const void* q, const void* k, const void* v,
+                         const void* q_idx, const void* k_idx, void* o, int32_t* idx_out,
+                         int32_t* cnt_out, uint8_t* flags_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
