@@ -9,7 +9,7 @@
 // One CTA per SM walks a static list of (query head, query block) items,
 // longest lists first.  The listed key blocks of consecutive items form one
 // stream indexed by a CTA-wide block counter g, so loads and products run
-// ahead across item boundaries.  10 warps:
+// ahead across item boundaries.  14 warps:
 //   warp 0     TMA producer: Q of item t into Q[t % 2]; K_j, V_j of block g
 //              into a 4-stage ring (positions 2g, 2g + 1).
 //   warp 1     TMEM owner and single-thread MMA issuer, in the order
@@ -17,11 +17,15 @@
 //                S(g)  = Q K_j^T        -> TMEM S[g % 2]
 //                PV(g) : O[t % 2] += P(g) V_j, with P(g) (bf16) read from the
 //                        first half of S[g % 2], where the softmax wrote it.
-//   warps 2-5  softmax: one query row per thread; S row -> running maximum
-//              (moved, and O rescaled in TMEM, only when it grows by more
-//              than 2^8) -> P; row sums handed to the epilogue per item.
-//   warps 6-9  epilogue: O[t % 2] / l -> global memory, overlapping the next
-//              item's products.
+//   warps 2-9  softmax: two warps per TMEM lane quadrant, each owning 64 of
+//              the 128 key columns of its 32 query rows; the row maximum is
+//              exchanged through shared memory (a 64-arrival mbarrier per
+//              quadrant, bounded wait), the running maximum is moved (and O rescaled in
+//              TMEM, each warp its half of the columns) only when it grows
+//              by more than 2^8; P is written back as bf16; the two partial
+//              row sums are handed to the epilogue per item.
+//   warps 10-13 epilogue: O[t % 2] / l -> global memory, overlapping the
+//              next item's products.
 // Every wait is bounded (2 s); on expiry the CTA records SBSA_ERR_TIMEOUT,
 // stops issuing, drains its copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -36,7 +40,7 @@ namespace {
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
@@ -48,11 +52,12 @@ struct PS {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int OFF_Q = 0;                            // Q[2]
   static constexpr int OFF_KV = 2 * Q_BYTES;                 // ring[kStages]
-  static constexpr int OFF_L = OFF_KV + kStages * KV_BYTES;  // row sums [2][BM]
-  static constexpr int OFF_BAR = OFF_L + 2 * BM * 4;
+  static constexpr int OFF_L = OFF_KV + kStages * KV_BYTES;  // row sums [item%2][half][BM]
+  static constexpr int OFF_MX = OFF_L + 4 * BM * 4;          // row max [block%2][half][BM]
+  static constexpr int OFF_BAR = OFF_MX + 4 * BM * 4;
   // q_full[2] q_free[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done[2]
-  // o_full[2] o_free[2] l_full[2] drain
-  static constexpr int NBARS = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 2 + 1;
+  // o_full[2] o_free[2] l_full[2] mx_ready[2][4] drain
+  static constexpr int NBARS = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 2 + 8 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S = 0;       // S[0], S[1]: 2 x BN columns
@@ -131,8 +136,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
   uint64_t* o_full = pv_done + 2;
   uint64_t* o_free = o_full + 2;
   uint64_t* l_full = o_free + 2;
-  uint64_t* drain = l_full + 2;
+  uint64_t* mx_ready = l_full + 2;  // [block % 2][quadrant]
+  uint64_t* drain = mx_ready + 8;
   float* l_buf = reinterpret_cast<float*>(smem + C::OFF_L);
+  float* mx_buf = reinterpret_cast<float*>(smem + C::OFF_MX);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   unsigned char* sQ = smem + C::OFF_Q;
@@ -146,11 +153,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
       mbar_init(&q_full[b], 1);
       mbar_init(&q_free[b], 1);
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&p_full[b], 256);
       mbar_init(&pv_done[b], 1);
       mbar_init(&o_full[b], 1);
       mbar_init(&o_free[b], 128);
-      mbar_init(&l_full[b], 128);
+      mbar_init(&l_full[b], 256);
+      for (int q = 0; q < 4; ++q) mbar_init(&mx_ready[b * 4 + q], 64);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -324,9 +332,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
         mbar_wait_bounded(drain, 0, &never, kTimeoutNs);
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // ================================================================ softmax
-    const int qd = warp & 3;
+    const int qd = warp & 3;             // TMEM lane quadrant
+    const int hf = (warp - 2) >> 2;      // which 64 key columns (and D/2 O columns)
     const int row = qd * 32 + lane;
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
     int g = 0;
@@ -334,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
     Item it;
     for (int t = 0; ok && load_item(p, t, it); ++t) {
       float m_run = -INFINITY, l_run = 0.f;
-      const uint32_t o_col = tmem + lane_base + C::TM_O + (t & 1) * D;
+      const uint32_t o_col = tmem + lane_base + C::TM_O + (t & 1) * D + hf * (D / 2);
       int b = 0;
       for (int r = 0; r < it.count; ++r) {
         const int j = it.list[r];
@@ -347,25 +356,34 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
           break;
         }
         tc_fence_after();
-        // pass 1: row maximum (64 columns at a time)
+        // this warp's 64 S columns, kept in registers
+        float a[32], bb[32];
+        tmem_ld32(s_col + hf * 64, a);
+        tmem_ld32(s_col + hf * 64 + 32, bb);
+        tmem_wait_ld();
+        const int c0 = hf * 64;  // key index of a[0] within the block
         float mx = -INFINITY;
+        if (diag) {
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 64) {
-          float a[32], bb[32];
-          tmem_ld32(s_col + c0, a);
-          tmem_ld32(s_col + c0 + 32, bb);
-          tmem_wait_ld();
-          if (diag) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c0 + c <= row) mx = fmaxf(mx, a[c]);
-              if (c0 + 32 + c <= row) mx = fmaxf(mx, bb[c]);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(a[c], bb[c]));
+          for (int c = 0; c < 32; ++c) {
+            if (c0 + c <= row) mx = fmaxf(mx, a[c]);
+            if (c0 + 32 + c <= row) mx = fmaxf(mx, bb[c]);
           }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(a[c], bb[c]));
         }
+        // exchange the half-row maxima with the partner warp; both warps have
+        // finished reading S, so P may then overwrite the first S columns
+        float* mxb = mx_buf + (g & 1) * 2 * BM;
+        mxb[hf * BM + row] = mx;
+        mbar_arrive(&mx_ready[(g & 1) * 4 + qd]);
+        if (!wait(&mx_ready[(g & 1) * 4 + qd], (g >> 1) & 1)) ok = false;
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+          ok = false;
+          break;
+        }
+        mx = fmaxf(mx, mxb[(hf ^ 1) * BM + row]);
         const float m_new = fmaxf(m_run, mx * p.scale_log2);
         if (b == 0) {
           m_run = m_new;
@@ -381,44 +399,35 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
           l_run *= alpha;
           m_run = m_new;
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            float o[32];
-            tmem_ld32(o_col + c0, o);
+          for (int oc = 0; oc < D / 2; oc += 16) {
+            float o[16];
+            tmem_ld16(o_col + oc, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] *= alpha;
-            tmem_st32(o_col + c0, o);
+            for (int c = 0; c < 16; ++c) o[c] *= alpha;
+            tmem_st16(o_col + oc, o);
           }
         }
-        // pass 2: P = exp2(S * scale - m) as bf16 over the first half of the
-        // S columns (step c0 reads S[c0, c0+64), writes P to [c0/2, c0/2+32),
-        // columns whose S values were already read)
+        // P = exp2(S * scale - m) as bf16: keys [c0, c0+64) -> columns [c0/2, c0/2+32)
         float lsum = 0.f;
+        uint32_t pk[32];
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 64) {
-          float a[32], bb[32];
-          tmem_ld32(s_col + c0, a);
-          tmem_ld32(s_col + c0 + 32, bb);
-          tmem_wait_ld();
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
-            float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
-            float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
-            float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
-            if (diag) {
-              if (c0 + c > row) p0 = 0.f;
-              if (c0 + c + 1 > row) p1 = 0.f;
-              if (c0 + 32 + c > row) p2 = 0.f;
-              if (c0 + 32 + c + 1 > row) p3 = 0.f;
-            }
-            lsum += (p0 + p1) + (p2 + p3);
-            pk[c >> 1] = pack_bf16x2(p0, p1);
-            pk[16 + (c >> 1)] = pack_bf16x2(p2, p3);
+        for (int c = 0; c < 32; c += 2) {
+          float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
+          float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
+          float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
+          float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
+          if (diag) {
+            if (c0 + c > row) p0 = 0.f;
+            if (c0 + c + 1 > row) p1 = 0.f;
+            if (c0 + 32 + c > row) p2 = 0.f;
+            if (c0 + 32 + c + 1 > row) p3 = 0.f;
           }
-          tmem_st32u(s_col + (c0 >> 1), pk);
+          lsum += (p0 + p1) + (p2 + p3);
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+          pk[16 + (c >> 1)] = pack_bf16x2(p2, p3);
         }
+        tmem_st32u(s_col + hf * 32, pk);
         l_run += lsum;
         tmem_wait_st();
         tc_fence_before();
@@ -427,13 +436,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
         ++b;
       }
       if (!ok) break;
-      // hand the row sum to the epilogue once it is done with item t - 2
+      // hand the partial row sum to the epilogue once it is done with item t - 2
       if (t >= 2 && !wait(&o_free[t & 1], ((t - 2) >> 1) & 1)) ok = false;
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         ok = false;
         break;
       }
-      l_buf[(t & 1) * BM + row] = (b > 0) ? l_run : 0.f;
+      l_buf[((t & 1) * 2 + hf) * BM + row] = (b > 0) ? l_run : 0.f;
       mbar_arrive(&l_full[t & 1]);
     }
     if (!ok && lane == 0 && !*abort_flag) fail(SBSA_ERR_TIMEOUT);
@@ -452,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
         break;
       }
       tc_fence_after();
-      const float l = l_buf[(t & 1) * BM + row];
+      const float l = l_buf[((t & 1) * 2 + 0) * BM + row] + l_buf[((t & 1) * 2 + 1) * BM + row];
       const float inv_l = (it.valid > 0 && l > 0.f) ? 1.f / l : 0.f;
       const int tok = it.i * BM + row;
       const bool store = tok < p.n;
