@@ -22,7 +22,7 @@
 //              exchanged through shared memory (a 64-arrival mbarrier per
 //              quadrant, bounded wait), the running maximum is moved (and O rescaled in
 //              TMEM, each warp its half of the columns) only when it grows
-//              by more than 2^8; P is written back as bf16; the two partial
+//              by more than 2^24; P is written back as bf16; the two partial
 //              row sums are handed to the epilogue per item.
 //   warps 10-13 epilogue: O[t % 2] / l -> global memory, overlapping the
 //              next item's products.
@@ -41,7 +41,10 @@ namespace {
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStages = 4;
 constexpr int kThreads = 448;
-constexpr float kRescaleLog2 = 8.0f;
+// The running maximum used for exp2 moves (and O is rescaled) only when the
+// row maximum exceeds it by more than 2^24: P stays below 2^24 in bf16 and
+// the fp32 row sums and O accumulators stay far from overflow.
+constexpr float kRescaleLog2 = 24.0f;
 
 template <int D>
 struct PS {
@@ -84,11 +87,15 @@ struct PSParams {
 struct Item {
   int i, h, g, count, valid;
   const int32_t* list;
+  int chunk_base;  // first list index held in chunk_val
+  int chunk_val;   // list[chunk_base + lane] (or -1 past the end)
 };
 
 // Item number t of this CTA (static round robin over the longest-first
-// order); `valid` counts the list entries inside [0, i].
-__device__ __forceinline__ bool load_item(const PSParams& p, int t, Item& it) {
+// order), read by a whole warp: each lane fetches one list entry, so up to
+// 32 entries cost one memory round trip.  `valid` counts the entries inside
+// [0, i].  Every lane of the warp must call this (and item_entry) together.
+__device__ __forceinline__ bool load_item(const PSParams& p, int t, Item& it, int lane) {
   const long long item = (long long)blockIdx.x + (long long)t * gridDim.x;
   if (item >= p.total) return false;
   it.i = p.nb - 1 - (int)(item / p.hq);
@@ -98,13 +105,25 @@ __device__ __forceinline__ bool load_item(const PSParams& p, int t, Item& it) {
   it.list = p.idx + ((size_t)hs * p.nb + it.i) * p.kmax;
   const int c = p.cnt[(size_t)hs * p.nb + it.i];
   it.count = c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
-  int v = 0;
-  for (int r = 0; r < it.count; ++r) {
-    const int j = it.list[r];
-    v += (j >= 0 && j <= it.i) ? 1 : 0;
+  it.chunk_base = 0;
+  it.chunk_val = lane < it.count ? it.list[lane] : -1;
+  int v = __popc(__ballot_sync(0xFFFFFFFFu, it.chunk_val >= 0 && it.chunk_val <= it.i));
+  for (int base = 32; base < it.count; base += 32) {
+    const int x = base + lane < it.count ? it.list[base + lane] : -1;
+    v += __popc(__ballot_sync(0xFFFFFFFFu, x >= 0 && x <= it.i));
   }
   it.valid = v;
   return true;
+}
+
+// List entry r of the item (uniform r across the warp).
+__device__ __forceinline__ int item_entry(Item& it, int r, int lane) {
+  const int base = r & ~31;
+  if (base != it.chunk_base) {
+    it.chunk_base = base;
+    it.chunk_val = base + lane < it.count ? it.list[base + lane] : -1;
+  }
+  return __shfl_sync(0xFFFFFFFFu, it.chunk_val, r & 31);
 }
 
 __device__ __forceinline__ bool valid_entry(const Item& it, int j) { return j >= 0 && j <= it.i; }
@@ -185,47 +204,65 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
     return mbar_wait_bounded(b, parity, abort_flag, kTimeoutNs);
   };
 
+  // Producer and MMA roles run as whole warps (list entries are fetched
+  // cooperatively); lane 0 issues the copies and products, and each wait's
+  // outcome is broadcast so the warp leaves a loop together.
+  auto warp_ok = [&](bool v) { return __shfl_sync(0xFFFFFFFFu, v, 0); };
+
   if (warp == 0) {
     // ================================================================ TMA
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
-      int pos = 0, t = 0, q_loaded = 0;
-      bool ok = true;
-      Item it;
-      for (; ok && load_item(p, t, it); ++t) {
-        const int qb = t & 1;
-        if (t >= 2 && !wait(&q_free[qb], ((t - 2) >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
-        for (int a = 0; a < C::NA_D; ++a)
-          tma_load_3d(sQ + qb * C::Q_BYTES + a * (BM * 128), &p.tm_q, &q_full[qb], a * 64,
-                      it.i * BM, it.h);
-        q_loaded = t + 1;
-        for (int r = 0; ok && r < it.count; ++r) {
-          const int j = it.list[r];
-          if (!valid_entry(it, j)) {
-            record(p.status, SBSA_ERR_DEVICE);
-            continue;
-          }
-          for (int half = 0; half < 2; ++half) {
-            const int st = pos % kStages;
-            if (!wait(&kv_empty[st], ((pos / kStages) & 1) ^ 1)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
-            const CUtensorMap* m = half ? &p.tm_v : &p.tm_k;
-            for (int a = 0; a < C::NA_D; ++a)
-              tma_load_3d(sKV + st * C::KV_BYTES + a * (BN * 128), m, &kv_full[st], a * 64,
-                          j * BN, it.g);
-            ++pos;
-          }
+    }
+    int pos = 0, t = 0, q_loaded = 0;
+    bool ok = true;
+    Item it;
+    for (; ok && load_item(p, t, it, lane); ++t) {
+      const int qb = t & 1;
+      bool good = true;
+      if (lane == 0) {
+        if (t >= 2) good = wait(&q_free[qb], ((t - 2) >> 1) & 1);
+        if (good) {
+          mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
+          for (int a = 0; a < C::NA_D; ++a)
+            tma_load_3d(sQ + qb * C::Q_BYTES + a * (BM * 128), &p.tm_q, &q_full[qb], a * 64,
+                        it.i * BM, it.h);
         }
       }
+      if (!warp_ok(good)) {
+        ok = false;
+        break;
+      }
+      q_loaded = t + 1;
+      for (int r = 0; ok && r < it.count; ++r) {
+        const int j = item_entry(it, r, lane);
+        if (!valid_entry(it, j)) {
+          if (lane == 0) record(p.status, SBSA_ERR_DEVICE);
+          continue;
+        }
+        for (int half = 0; half < 2; ++half) {
+          const int st = pos % kStages;
+          if (lane == 0) {
+            good = wait(&kv_empty[st], ((pos / kStages) & 1) ^ 1);
+            if (good) {
+              mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
+              const CUtensorMap* m = half ? &p.tm_v : &p.tm_k;
+              for (int a = 0; a < C::NA_D; ++a)
+                tma_load_3d(sKV + st * C::KV_BYTES + a * (BN * 128), m, &kv_full[st], a * 64,
+                            j * BN, it.g);
+            }
+          }
+          if (!warp_ok(good)) {
+            ok = false;
+            break;
+          }
+          ++pos;
+        }
+      }
+    }
+    if (lane == 0) {
       volatile int never = 0;
       const int first = pos > kStages ? pos - kStages : 0;
       if (!ok) {
@@ -245,85 +282,94 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
     }
   } else if (warp == 1) {
     // ================================================================ MMA
-    if (lane == 0) {
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t kv_base = smem_u32(sKV);
-      struct Pending {
-        int g, t, b, last;  // block counter, item, block within item, last of item
-      };
-      Pending prev{0, 0, 0, 0};
-      bool have_prev = false, ok = true;
-      auto issue_pv = [&](const Pending& pv) -> bool {
-        if (!wait(&p_full[pv.g & 1], (pv.g >> 1) & 1)) return false;
-        if (pv.b == 0 && pv.t >= 2 && !wait(&o_free[pv.t & 1], ((pv.t - 2) >> 1) & 1))
-          return false;
-        const int vpos = 2 * pv.g + 1;
-        const int st = vpos % kStages;
-        if (!wait(&kv_full[st], (vpos / kStages) & 1)) return false;
-        tc_fence_after();
-        const uint32_t v_base = kv_base + st * C::KV_BYTES;
-        const uint32_t a_col = tmem + C::TM_S + (pv.g & 1) * BN;
-        const uint32_t o_col = tmem + C::TM_O + (pv.t & 1) * D;
+    const uint32_t q_base = smem_u32(sQ);
+    const uint32_t kv_base = smem_u32(sKV);
+    struct Pending {
+      int g, t, b, last;  // block counter, item, block within item, last of item
+    };
+    Pending prev{0, 0, 0, 0};
+    bool have_prev = false, ok = true;
+    // lane 0 only
+    auto issue_pv = [&](const Pending& pv) -> bool {
+      if (!wait(&p_full[pv.g & 1], (pv.g >> 1) & 1)) return false;
+      if (pv.b == 0 && pv.t >= 2 && !wait(&o_free[pv.t & 1], ((pv.t - 2) >> 1) & 1))
+        return false;
+      const int vpos = 2 * pv.g + 1;
+      const int st = vpos % kStages;
+      if (!wait(&kv_full[st], (vpos / kStages) & 1)) return false;
+      tc_fence_after();
+      const uint32_t v_base = kv_base + st * C::KV_BYTES;
+      const uint32_t a_col = tmem + C::TM_S + (pv.g & 1) * BN;
+      const uint32_t o_col = tmem + C::TM_O + (pv.t & 1) * D;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = smem_desc(v_base + kk * 16 * 128, BN * 128, 1024);
-          umma_f16_ts(o_col, a_col + kk * 8, bd, C::IDESC_O, (pv.b > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < BN / 16; ++kk) {
+        const uint64_t bd = smem_desc(v_base + kk * 16 * 128, BN * 128, 1024);
+        umma_f16_ts(o_col, a_col + kk * 8, bd, C::IDESC_O, (pv.b > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&kv_empty[st]);
+      umma_commit(&pv_done[pv.g & 1]);
+      if (pv.last) umma_commit(&o_full[pv.t & 1]);
+      return true;
+    };
+    int g = 0, t = 0;
+    Item it;
+    for (; ok && load_item(p, t, it, lane); ++t) {
+      const int qb = t & 1;
+      bool good = true;
+      if (lane == 0) {
+        good = wait(&q_full[qb], (t >> 1) & 1);
+        if (good) {
+          tc_fence_after();
+          if (it.valid == 0) {
+            // nothing to multiply: release Q; the epilogue writes zeros
+            umma_commit(&q_free[qb]);
+            umma_commit(&o_full[qb]);
+          }
         }
-        umma_commit(&kv_empty[st]);
-        umma_commit(&pv_done[pv.g & 1]);
-        if (pv.last) umma_commit(&o_full[pv.t & 1]);
-        return true;
-      };
-      int g = 0, t = 0;
-      Item it;
-      for (; ok && load_item(p, t, it); ++t) {
-        const int qb = t & 1;
-        if (!wait(&q_full[qb], (t >> 1) & 1)) {
+      }
+      if (!warp_ok(good)) {
+        ok = false;
+        break;
+      }
+      if (it.valid == 0) continue;
+      int b = 0;
+      for (int r = 0; r < it.count; ++r) {
+        const int j = item_entry(it, r, lane);
+        if (!valid_entry(it, j)) continue;
+        const bool last = (b == it.valid - 1);
+        if (lane == 0) {
+          const int kpos = 2 * g;
+          const int st = kpos % kStages;
+          good = wait(&kv_full[st], (kpos / kStages) & 1);
+          if (good) {
+            tc_fence_after();
+            const uint32_t qa = q_base + qb * C::Q_BYTES;
+            const uint32_t ka = kv_base + st * C::KV_BYTES;
+            const uint32_t s_col = tmem + C::TM_S + (g & 1) * BN;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int kb = kk * 32;
+              const uint64_t ad = smem_desc(qa + (kb / 128) * (BM * 128) + (kb % 128), 16, 1024);
+              const uint64_t bd = smem_desc(ka + (kb / 128) * (BN * 128) + (kb % 128), 16, 1024);
+              umma_f16_ss(s_col, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&kv_empty[st]);
+            umma_commit(&s_full[g & 1]);
+            if (last) umma_commit(&q_free[qb]);
+            if (have_prev) good = issue_pv(prev);
+          }
+        }
+        if (!warp_ok(good)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (it.valid == 0) {
-          // nothing to multiply: release Q; the epilogue writes zeros
-          umma_commit(&q_free[qb]);
-          umma_commit(&o_full[qb]);
-          continue;
-        }
-        int b = 0;
-        for (int r = 0; r < it.count; ++r) {
-          const int j = it.list[r];
-          if (!valid_entry(it, j)) continue;
-          const int kpos = 2 * g;
-          const int st = kpos % kStages;
-          if (!wait(&kv_full[st], (kpos / kStages) & 1)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t qa = q_base + qb * C::Q_BYTES;
-          const uint32_t ka = kv_base + st * C::KV_BYTES;
-          const uint32_t s_col = tmem + C::TM_S + (g & 1) * BN;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int kb = kk * 32;
-            const uint64_t ad = smem_desc(qa + (kb / 128) * (BM * 128) + (kb % 128), 16, 1024);
-            const uint64_t bd = smem_desc(ka + (kb / 128) * (BN * 128) + (kb % 128), 16, 1024);
-            umma_f16_ss(s_col, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&kv_empty[st]);
-          umma_commit(&s_full[g & 1]);
-          const bool last = (b == it.valid - 1);
-          if (last) umma_commit(&q_free[qb]);
-          if (have_prev && !issue_pv(prev)) {
-            ok = false;
-            break;
-          }
-          prev = Pending{g, t, b, last ? 1 : 0};
-          have_prev = true;
-          ++g;
-          ++b;
-        }
+        prev = Pending{g, t, b, last ? 1 : 0};
+        have_prev = true;
+        ++g;
+        ++b;
       }
+    }
+    if (lane == 0) {
       if (ok && have_prev) ok = issue_pv(prev);
       if (!ok) {
         if (!*abort_flag) fail(SBSA_ERR_TIMEOUT);
@@ -341,12 +387,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
     int g = 0;
     bool ok = true;
     Item it;
-    for (int t = 0; ok && load_item(p, t, it); ++t) {
+    for (int t = 0; ok && load_item(p, t, it, lane); ++t) {
       float m_run = -INFINITY, l_run = 0.f;
       const uint32_t o_col = tmem + lane_base + C::TM_O + (t & 1) * D + hf * (D / 2);
       int b = 0;
       for (int r = 0; r < it.count; ++r) {
-        const int j = it.list[r];
+        const int j = item_entry(it, r, lane);
         if (!valid_entry(it, j)) continue;
         const bool diag = (j == it.i);
         const uint32_t s_col = tmem + lane_base + C::TM_S + (g & 1) * BN;
@@ -453,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
     bool ok = true;
     Item it;
-    for (int t = 0; ok && load_item(p, t, it); ++t) {
+    for (int t = 0; ok && load_item(p, t, it, lane); ++t) {
       if (!wait(&l_full[t & 1], (t >> 1) & 1)) ok = false;
       if (ok && !wait(&o_full[t & 1], (t >> 1) & 1)) ok = false;
       if (!__all_sync(0xFFFFFFFFu, ok)) {

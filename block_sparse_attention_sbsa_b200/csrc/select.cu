@@ -12,10 +12,12 @@
 // rescue branch through the block radius, each with its own threshold, masks
 // united.  "MiniMax presenta MSA": one selection per GQA group.
 //
-// Layout of one CTA: R consecutive query blocks of one selection head.
-// Phase 1 computes their scores against every earlier key block into shared
-// memory (fp32 FMA, key-centroid chunks staged in shared memory so each
-// centroid is read from L2 once per CTA).  Phase 2 gives each row to a warp:
+// Layout of one CTA: R (up to 16) consecutive query blocks of one selection
+// head.  Phase 1 computes their scores against every earlier key block into
+// shared memory: each thread streams whole key-centroid rows from L2 in
+// 16-byte pieces and dots them with the R pooled queries held in shared
+// memory (fp32 FMA; each centroid row is read once per CTA).  Phase 2 gives
+// each row to a warp:
 // exact radix selection on order-preserving 32-bit keys (ties resolved by the
 // lower block id), 64-bit fixed-point mass histograms for the cumulative-mass
 // rule (deterministic sums), double-precision mean/std for the gate, then a
@@ -29,8 +31,8 @@ namespace {
 
 constexpr int kSelThreads = 256;
 constexpr int kWarps = kSelThreads / 32;
-constexpr int kJC = 128;      // candidate key blocks per scoring chunk
 constexpr int kMaxWalk = 24;  // ranked-walk steps before the radix fallback
+constexpr int kHistBytes = kWarps * 256 * 8;  // one 256-bin 64-bit histogram per warp
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
@@ -234,13 +236,11 @@ __device__ uint32_t radix_select_mass(const float* s, int n, float smax, double 
 template <int DS, int R>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_constant__ SelectArgs a,
                                                             int score_stride) {
-  static_assert(R % 2 == 0 && R <= 8, "rows per CTA");
-  constexpr int CS = DS + 4;  // padded centroid row stride (floats)
+  static_assert(R <= 16, "rows per CTA");
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* qs = reinterpret_cast<float*>(smem_raw);       // [R][DS]
-  float* cs = qs + R * DS;                              // [kJC][CS]  (phase 1)
-  float* sc = cs + kJC * CS;                            // [R][score_stride]
-  unsigned char* hist_base = reinterpret_cast<unsigned char*>(cs);  // phase 2 reuse
+  float* qs = reinterpret_cast<float*>(smem_raw);                 // [R][DS]
+  unsigned char* hist_base = reinterpret_cast<unsigned char*>(qs + R * DS);  // phase 2
+  float* sc = reinterpret_cast<float*>(hist_base + kHistBytes);   // [R][score_stride]
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -257,43 +257,32 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
     const int r = e / DS;
     qs[e] = (r < rows) ? a.qc[((size_t)hs * a.nb + i0 + r) * DS + (e % DS)] : 0.f;
   }
+  __syncthreads();
 
-  // ---- phase 1: scores ----
-  constexpr int RH = R / 2;
-  const int tj = tid % kJC;
-  const int th = tid / kJC;
+  // ---- phase 1: scores.  Each thread owns candidate blocks j = tid + 256u
+  // and streams their centroid rows (fp32) from L2 in 16-byte pieces, dotting
+  // each piece with the R pooled queries read from shared memory (every lane
+  // reads the same address: one broadcast per row).
   const float* kc = a.kc + (size_t)g * a.nb * DS;
-  for (int j0 = 0; j0 < jend; j0 += kJC) {
-    __syncthreads();
-    for (int e = tid * 4; e < kJC * DS; e += kSelThreads * 4) {
-      const int jj = e / DS, col = e % DS;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + jj < jend) v = *reinterpret_cast<const float4*>(kc + (size_t)(j0 + jj) * DS + col);
-      *reinterpret_cast<float4*>(cs + jj * CS + col) = v;
-    }
-    __syncthreads();
-    float acc[RH];
+  for (int j = tid; j < jend; j += kSelThreads) {
+    const float4* crow = reinterpret_cast<const float4*>(kc + (size_t)j * DS);
+    float acc[R];
 #pragma unroll
-    for (int r = 0; r < RH; ++r) acc[r] = 0.f;
-    const float* crow = cs + tj * CS;
-    const float* qrow = qs + th * RH * DS;
+    for (int r = 0; r < R; ++r) acc[r] = 0.f;
 #pragma unroll 4
-    for (int k = 0; k < DS; k += 4) {
-      const float4 c4 = *reinterpret_cast<const float4*>(crow + k);
+    for (int k4 = 0; k4 < DS / 4; ++k4) {
+      const float4 c4 = __ldg(crow + k4);
 #pragma unroll
-      for (int r = 0; r < RH; ++r) {
-        const float4 q4 = *reinterpret_cast<const float4*>(qrow + r * DS + k);
+      for (int r = 0; r < R; ++r) {
+        const float4 q4 = *reinterpret_cast<const float4*>(qs + r * DS + 4 * k4);
         acc[r] = fmaf(q4.x, c4.x, acc[r]);
         acc[r] = fmaf(q4.y, c4.y, acc[r]);
         acc[r] = fmaf(q4.z, c4.z, acc[r]);
         acc[r] = fmaf(q4.w, c4.w, acc[r]);
       }
     }
-    const int j = j0 + tj;
-    if (j < jend) {
 #pragma unroll
-      for (int r = 0; r < RH; ++r) sc[(th * RH + r) * score_stride + j] = acc[r] * a.score_scale;
-    }
+    for (int r = 0; r < R; ++r) sc[r * score_stride + j] = acc[r] * a.score_scale;
   }
   __syncthreads();
 
@@ -483,9 +472,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
 template <int DS, int R>
 cudaError_t launch_rows(const SelectArgs& a, cudaStream_t stream) {
   const int stride = (a.nb + 3) & ~3;
-  const size_t smem = (size_t)(R * DS + kJC * (DS + 4) + R * stride) * sizeof(float);
-  const size_t hist_need = (size_t)kWarps * 256 * 8;
-  if (hist_need > (size_t)kJC * (DS + 4) * sizeof(float)) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)R * DS * 4 + kHistBytes + (size_t)R * stride * 4;
   auto kern = select_kernel<DS, R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -498,13 +485,14 @@ cudaError_t launch_rows(const SelectArgs& a, cudaStream_t stream) {
 
 template <int DS>
 cudaError_t launch_ds(const SelectArgs& a, cudaStream_t stream) {
-  // rows per CTA: as many as the score rows fit next to the centroid chunk
-  const size_t fixed = (size_t)kJC * (DS + 4) * 4;
-  const size_t budget = 220 * 1024;
+  // rows per CTA: as many (up to 16) as the score rows allow in shared memory;
+  // more rows per CTA means fewer reads of each centroid row from L2
+  const size_t budget = 200 * 1024;
   const size_t row = (size_t)((a.nb + 3) & ~3) * 4 + DS * 4;
-  if (fixed + 8 * row <= budget) return launch_rows<DS, 8>(a, stream);
-  if (fixed + 4 * row <= budget) return launch_rows<DS, 4>(a, stream);
-  if (fixed + 2 * row <= budget) return launch_rows<DS, 2>(a, stream);
+  if (kHistBytes + 16 * row <= budget) return launch_rows<DS, 16>(a, stream);
+  if (kHistBytes + 8 * row <= budget) return launch_rows<DS, 8>(a, stream);
+  if (kHistBytes + 4 * row <= budget) return launch_rows<DS, 4>(a, stream);
+  if (kHistBytes + 2 * row <= budget) return launch_rows<DS, 2>(a, stream);
   return cudaErrorInvalidValue;
 }
 
