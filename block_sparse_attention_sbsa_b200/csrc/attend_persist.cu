@@ -22,7 +22,7 @@
 //              exchanged through shared memory (a 64-arrival mbarrier per
 //              quadrant, bounded wait), the running maximum is moved (and O rescaled in
 //              TMEM, each warp its half of the columns) only when it grows
-//              by more than 2^24; P is written back as bf16; the two partial
+//              by more than 2^8; P is written back as bf16; the two partial
 //              row sums are handed to the epilogue per item.
 //   warps 10-13 epilogue: O[t % 2] / l -> global memory, overlapping the
 //              next item's products.
@@ -42,9 +42,8 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStages = 4;
 constexpr int kThreads = 448;
 // The running maximum used for exp2 moves (and O is rescaled) only when the
-// row maximum exceeds it by more than 2^24: P stays below 2^24 in bf16 and
-// the fp32 row sums and O accumulators stay far from overflow.
-constexpr float kRescaleLog2 = 24.0f;
+// row maximum exceeds it by more than 2^8 (P stays below 256).
+constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
 struct PS {
