@@ -531,13 +531,20 @@ cudaError_t launch_wait_probe(uint64_t timeout_ns, int* status, cudaStream_t str
 }
 
 int launch_attend(const AttendArgs& a, cudaStream_t stream) {
-  static const bool single = [] {
+  // 0: automatic, 1: pair, 2: persistent, 3: single
+  static const int forced = [] {
     const char* e = std::getenv("SBSA_ATTEND_KERNEL");
-    return e && std::strcmp(e, "single") == 0;
+    if (!e) return 0;
+    if (std::strcmp(e, "pair") == 0) return 1;
+    if (std::strcmp(e, "persistent") == 0) return 2;
+    if (std::strcmp(e, "single") == 0) return 3;
+    return 0;
   }();
-  if (!single && a.dtype == SBSA_BF16 && a.block == 128 && (a.d == 128 || a.d == 64))
-    return launch_attend_persistent(a, stream);
-  return launch_attend_single(a, stream);
+  const bool big = a.dtype == SBSA_BF16 && a.block == 128 && (a.d == 128 || a.d == 64);
+  const bool pairable = big && (a.hq / a.hkv) % 2 == 0;
+  if (forced == 3 || !big) return launch_attend_single(a, stream);
+  if (forced == 2 || !pairable) return launch_attend_persistent(a, stream);
+  return launch_attend_pair(a, stream);
 }
 
 int launch_attend_single(const AttendArgs& a, cudaStream_t stream) {

@@ -59,10 +59,15 @@ struct AttendArgs {
 };
 
 // Returns an SBSA_* code (SBSA_ERR_CUDA on launch/driver failure).  bf16
-// with 128-token blocks runs the persistent pipelined kernel unless the
-// environment variable SBSA_ATTEND_KERNEL is "single"; every other
-// combination runs the one-tile-per-CTA kernel.
+// with 128-token blocks runs the head-pair kernel when the GQA group has an
+// even number of query heads, else the persistent kernel; every other
+// combination runs the one-tile-per-CTA kernel.  The environment variable
+// SBSA_ATTEND_KERNEL ("pair", "persistent", "single") overrides the choice
+// where the requested kernel supports the arguments.
 int launch_attend(const AttendArgs& a, cudaStream_t stream);
+
+// The head-pair kernel (bf16, B = 128, d in {64, 128}, even group size).
+int launch_attend_pair(const AttendArgs& a, cudaStream_t stream);
 
 // The one-tile-per-CTA kernel (every supported dtype / block / d).
 int launch_attend_single(const AttendArgs& a, cudaStream_t stream);

@@ -307,9 +307,11 @@ def test_bounded_wait_reports_timeout_and_context_survives(sb):
     assert mx <= PT.MAX_ABS
 
 
-def test_single_tile_kernel_matches_oracle_too(sb):
-    """The one-tile-per-CTA attention kernel (selected by SBSA_ATTEND_KERNEL)
-    on the 128-token-block workloads, in a child process."""
+@pytest.mark.parametrize("kernel", ["single", "persistent"])
+def test_alternative_attention_kernels_match_oracle_too(sb, kernel):
+    """The one-tile-per-CTA and the persistent one-tile-stream attention
+    kernels (selected by SBSA_ATTEND_KERNEL) on the 128-token-block
+    workloads, in a child process."""
     import os
     import subprocess
     import sys
@@ -327,9 +329,44 @@ def test_single_tile_kernel_matches_oracle_too(sb):
         "    assert sbsa.get_status() == sbsa.OK\n"
         "    mx, mean = PT.output_errors(o.float().cpu().numpy(), ref['o'])\n"
         "    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (name, mx, mean)\n"
-        "print('single ok')\n")
+        "print('kernel ok')\n")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, SBSA_ATTEND_KERNEL="single")
+    env = dict(os.environ, SBSA_ATTEND_KERNEL=kernel)
     r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True,
                        text=True, timeout=600)
-    assert r.returncode == 0 and "single ok" in r.stdout, r.stdout + r.stderr
+    assert r.returncode == 0 and "kernel ok" in r.stdout, r.stdout + r.stderr
+
+
+@pytest.mark.parametrize("case", [
+    dict(select_mode="cummass", mass_threshold=1.0),                      # keep everything
+    dict(select_mode="cummass", mass_threshold=0.5, rescue_tau=-1e30),    # rescue everything
+    dict(top_k=1),                                                        # one past block
+    dict(top_k=2, gate_margin=1e6),                                       # gate always fires
+    dict(top_k=2, gate_margin=0.0),                                       # gate never fires
+    dict(top_k=3, n_q_heads=2, n_kv_heads=2),                             # one head per group
+])
+def test_degenerate_selection_parameters(sb, case):
+    n, b, d = 1200, 128, 128
+    hq = case.pop("n_q_heads", 4)
+    hk = case.pop("n_kv_heads", 2)
+    q, k, v = _random_case(hq, hk, n, d, b, "bf16", 17)
+    p = sb.make_params(n_q_heads=hq, n_kv_heads=hk, seq_len=n, head_dim=d, block_size=b, **case)
+    o, idx, cnt, flags = sb.prefill(p, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    assert sb.get_status() == sb.OK
+    mode = case.get("select_mode", "topk")
+    ref = O.prefill(q, k, v, block=b, mode=mode, top_k_=case.get("top_k", 0),
+                    mass=case.get("mass_threshold", 0.0), margin=case.get("gate_margin"),
+                    tau=case.get("rescue_tau"), max_blocks=p.max_blocks)
+    w = W.Workload("case", "gqa", hq, hk, n, d, b, "bf16", mode, top_k=case.get("top_k", 0),
+                   mass_threshold=case.get("mass_threshold", 0.0),
+                   rescue_tau=case.get("rescue_tau"), gate_margin=case.get("gate_margin"))
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    rows = [(h, i) for h in range(hq) for i in range(O.n_blocks(n, b))]
+    PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], rows, ref["qbar"], ref["c"], ref["r"], w,
+                     lambda hs: hs // (hq // hk))
+    if mode == "cummass" and (case.get("mass_threshold") == 1.0 or case.get("rescue_tau")):
+        assert np.array_equal(cnt, ref["cnt"])
+        assert all(cnt[0, i] == i + 1 for i in range(O.n_blocks(n, b)))
+    mx, mean = PT.output_errors(o.float().cpu().numpy(), ref["o"])
+    assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
