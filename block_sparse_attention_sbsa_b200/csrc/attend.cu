@@ -541,7 +541,9 @@ int launch_attend(const AttendArgs& a, cudaStream_t stream) {
     return 0;
   }();
   const bool big = a.dtype == SBSA_BF16 && a.block == 128 && (a.d == 128 || a.d == 64);
-  const bool pairable = big && (a.hq / a.hkv) % 2 == 0;
+  // The pair kernel pays off when the two heads' lists coincide (one list
+  // per GQA group); with per-head lists the overlap is too small.
+  const bool pairable = big && a.group_shared && (a.hq / a.hkv) % 2 == 0;
   if (forced == 3 || !big) return launch_attend_single(a, stream);
   if (forced == 2 || !pairable) return launch_attend_persistent(a, stream);
   return launch_attend_pair(a, stream);

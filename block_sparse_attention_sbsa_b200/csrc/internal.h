@@ -59,9 +59,9 @@ struct AttendArgs {
 };
 
 // Returns an SBSA_* code (SBSA_ERR_CUDA on launch/driver failure).  bf16
-// with 128-token blocks runs the head-pair kernel when the GQA group has an
-// even number of query heads, else the persistent kernel; every other
-// combination runs the one-tile-per-CTA kernel.  The environment variable
+// with 128-token blocks runs the head-pair kernel for lists shared by a GQA
+// group with an even number of query heads, else the persistent kernel;
+// every other combination runs the one-tile-per-CTA kernel.  The environment variable
 // SBSA_ATTEND_KERNEL ("pair", "persistent", "single") overrides the choice
 // where the requested kernel supports the arguments.
 int launch_attend(const AttendArgs& a, cudaStream_t stream);

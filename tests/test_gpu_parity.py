@@ -307,10 +307,10 @@ def test_bounded_wait_reports_timeout_and_context_survives(sb):
     assert mx <= PT.MAX_ABS
 
 
-@pytest.mark.parametrize("kernel", ["single", "persistent"])
+@pytest.mark.parametrize("kernel", ["single", "persistent", "pair"])
 def test_alternative_attention_kernels_match_oracle_too(sb, kernel):
-    """The one-tile-per-CTA and the persistent one-tile-stream attention
-    kernels (selected by SBSA_ATTEND_KERNEL) on the 128-token-block
+    """Each attention kernel forced by SBSA_ATTEND_KERNEL (one tile per CTA,
+    persistent one-tile stream, head pairs) on the 128-token-block
     workloads, in a child process."""
     import os
     import subprocess
