@@ -333,3 +333,65 @@ def attended_pairs(p: Params, cnt: torch.Tensor) -> int:
         c = c.repeat_interleave(p.n_q_heads // p.n_kv_heads, dim=0)
     past = ((c - 1).clamp(min=0) * rows.view(1, -1) * b).sum()
     return int(past + (diag.view(1, -1) * (c > 0)).sum())
+
+
+class PrefillPipeline:
+    """Prefills from and to pinned host buffers with copies overlapped.
+
+    Each submitted request copies its inputs host -> device, runs the
+    prefill (one sbsa_prefill call) and copies O device -> host.  Two device
+    buffer sets and three streams let the next request's input copy and the
+    previous request's output copy run while the current prefill computes;
+    the order of requests is preserved.  Host tensors must be pinned and
+    must stay untouched until `synchronize()` (or the request two
+    submissions later) has completed.
+    """
+
+    def __init__(self, p: Params, device="cuda", with_index: bool = False):
+        self.p = p
+        self.device = torch.device(device)
+        dt = _TORCH_DT[p.dtype]
+        shapes = {"q": (p.n_q_heads, p.seq_len, p.head_dim),
+                  "k": (p.n_kv_heads, p.seq_len, p.head_dim),
+                  "v": (p.n_kv_heads, p.seq_len, p.head_dim)}
+        if p.index_dim:
+            shapes["q_idx"] = (p.n_q_heads, p.seq_len, p.index_dim)
+            shapes["k_idx"] = (p.n_kv_heads, p.seq_len, p.index_dim)
+        self.bufs = [{k: torch.empty(s, dtype=dt, device=self.device) for k, s in shapes.items()}
+                     for _ in range(2)]
+        self.outs = [torch.empty(shapes["q"], dtype=dt, device=self.device) for _ in range(2)]
+        self.calls = [Prefill(p, device=self.device, keep_lists=False) for _ in range(2)]
+        self.h2d = torch.cuda.Stream(self.device)
+        self.comp = torch.cuda.Stream(self.device)
+        self.d2h = torch.cuda.Stream(self.device)
+        self.in_free = [torch.cuda.Event() for _ in range(2)]    # compute done with inputs
+        self.in_ready = [torch.cuda.Event() for _ in range(2)]   # inputs copied
+        self.out_ready = [torch.cuda.Event() for _ in range(2)]  # prefill done
+        self.out_free = [torch.cuda.Event() for _ in range(2)]   # output copied back
+        self.n = 0
+
+    def submit(self, host_in: dict, host_out: torch.Tensor):
+        s = self.n % 2
+        bufs, out = self.bufs[s], self.outs[s]
+        if self.n >= 2:
+            self.h2d.wait_event(self.in_free[s])
+        with torch.cuda.stream(self.h2d):
+            for name, dev in bufs.items():
+                dev.copy_(host_in[name], non_blocking=True)
+            self.in_ready[s].record(self.h2d)
+        self.comp.wait_event(self.in_ready[s])
+        if self.n >= 2:
+            self.comp.wait_event(self.out_free[s])
+        self.calls[s](bufs["q"], bufs["k"], bufs["v"], bufs.get("q_idx"), bufs.get("k_idx"),
+                      out=out, stream=self.comp)
+        self.in_free[s].record(self.comp)
+        self.out_ready[s].record(self.comp)
+        self.d2h.wait_event(self.out_ready[s])
+        with torch.cuda.stream(self.d2h):
+            host_out.copy_(out, non_blocking=True)
+            self.out_free[s].record(self.d2h)
+        self.n += 1
+
+    def synchronize(self):
+        for st in (self.h2d, self.comp, self.d2h):
+            st.synchronize()

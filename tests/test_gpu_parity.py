@@ -370,3 +370,25 @@ def test_degenerate_selection_parameters(sb, case):
         assert all(cnt[0, i] == i + 1 for i in range(O.n_blocks(n, b)))
     mx, mean = PT.output_errors(o.float().cpu().numpy(), ref["o"])
     assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
+
+
+def test_prefill_pipeline_from_host_buffers(sb):
+    """PrefillPipeline: pinned host inputs -> device -> prefill -> pinned host
+    output, three requests in flight order, each equal to a plain prefill."""
+    w = W.SMALL["gqa_small"]
+    p = sb.params_for(w)
+    pipe = sb.PrefillPipeline(p)
+    reqs, outs = [], []
+    for r in range(3):
+        data = W.generate(w.scaled(seed=w.seed + 50 + r), "cpu")
+        host = {k: data[k].pin_memory() for k in ("q", "k", "v")}
+        out = torch.empty(data["q"].shape, dtype=data["q"].dtype).pin_memory()
+        pipe.submit(host, out)
+        reqs.append(host)
+        outs.append(out)
+    pipe.synchronize()
+    assert sb.get_status() == sb.OK
+    for host, out in zip(reqs, outs):
+        ref, _, _, _ = sb.prefill(p, host["q"].cuda(), host["k"].cuda(), host["v"].cuda())
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref.cpu())
