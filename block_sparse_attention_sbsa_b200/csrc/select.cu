@@ -33,6 +33,7 @@ constexpr int kSelThreads = 256;
 constexpr int kWarps = kSelThreads / 32;
 constexpr int kMaxWalk = 24;  // ranked-walk steps before the radix fallback
 constexpr int kHistBytes = kWarps * 256 * 8;  // one 256-bin 64-bit histogram per warp
+constexpr int kShortCap = 256;                // short-list keys (second half of a warp's area)
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
@@ -82,10 +83,11 @@ __device__ __forceinline__ uint32_t warp_max_u(uint32_t v) {
   return v;
 }
 
-// Key of descending rank `want` (0-based) among fkey(s[0..n)).  *n_gt gets
-// the number of keys strictly greater, *n_eq the number equal to it.
-__device__ uint32_t radix_select(const float* s, int n, int want, uint32_t* hist, int* n_gt,
-                                 int* n_eq) {
+// Key of descending rank `want` (0-based) among key(0..n).  *n_gt gets the
+// number of keys strictly greater, *n_eq the number equal to it.
+template <typename KeyAt>
+__device__ uint32_t radix_select_keys(KeyAt key_at, int n, int want, uint32_t* hist, int* n_gt,
+                                      int* n_eq) {
   const int lane = threadIdx.x & 31;
   uint32_t prefix = 0, pmask = 0;
   uint32_t rank = (uint32_t)want, above = 0, eq = 0;
@@ -95,7 +97,7 @@ __device__ uint32_t radix_select(const float* s, int n, int want, uint32_t* hist
     for (int base = 0; base < n; base += 32) {
       const int j = base + lane;
       const bool in = j < n;
-      const uint32_t u = in ? fkey(s[j]) : 0u;
+      const uint32_t u = in ? key_at(j) : 0u;
       const bool match = in && ((u & pmask) == prefix);
       const uint32_t bin = (u >> shift) & 0xFFu;
       const unsigned act = __ballot_sync(0xFFFFFFFFu, match);
@@ -147,6 +149,58 @@ __device__ uint32_t radix_select(const float* s, int n, int want, uint32_t* hist
   *n_gt = (int)above;
   *n_eq = (int)eq;
   return prefix;
+}
+
+__device__ __forceinline__ uint32_t radix_select(const float* s, int n, int want, uint32_t* hist,
+                                                 int* n_gt, int* n_eq) {
+  return radix_select_keys([s](int j) { return fkey(s[j]); }, n, want, hist, n_gt, n_eq);
+}
+
+// Top-k cut through a short list.  Each lane keeps its T largest keys; the
+// (need)-th largest of those 32*T values is a lower bound of the row's
+// (need)-th largest key (at least `need` row keys reach it), so every key of
+// rank < need is among the keys >= the bound.  Those are compacted into
+// `buf` (at most `cap`) and the exact cut is taken there.  Returns false
+// (nothing computed) when the short list would overflow `buf`.
+template <int T>
+__device__ bool topk_short(const float* s, int n, int need, uint32_t* hist, uint32_t* buf, int cap,
+                           int* cnt_out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t top[T];
+#pragma unroll
+  for (int q = 0; q < T; ++q) top[q] = 0u;
+  for (int j = lane; j < n; j += 32) {
+    uint32_t u = fkey(s[j]);
+#pragma unroll
+    for (int q = 0; q < T; ++q) {  // insertion into the descending list
+      const uint32_t hi = max(top[q], u), lo = min(top[q], u);
+      top[q] = hi;
+      u = lo;
+    }
+  }
+  // the bound: rank need-1 among the 32*T lane values (absent values are 0,
+  // below every real key, and never reach rank need-1 while need <= n)
+#pragma unroll
+  for (int q = 0; q < T; ++q) buf[q * 32 + lane] = top[q];
+  __syncwarp();
+  int g, e;
+  const uint32_t bound = radix_select_keys([buf](int j) { return buf[j]; }, 32 * T, need - 1,
+                                           hist, &g, &e);
+  __syncwarp();
+  // compact the keys at or above the bound
+  int m = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = j < n ? fkey(s[j]) : 0u;
+    const bool keep = j < n && u >= bound;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
+    const int at = m + __popc(bal & ((1u << lane) - 1u));
+    if (keep && at < cap) buf[at] = u;
+    m += __popc(bal);
+  }
+  __syncwarp();
+  *cnt_out = m;
+  return m <= cap;
 }
 
 // Fixed-point probability of a candidate: softmax weight scaled by 2^60.
@@ -289,7 +343,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
   // ---- phase 2: one warp per row ----
   unsigned long long* hist64 =
       reinterpret_cast<unsigned long long*>(hist_base) + (size_t)warp * 256;
-  uint32_t* hist32 = reinterpret_cast<uint32_t*>(hist64);
+  uint32_t* hist32 = reinterpret_cast<uint32_t*>(hist64);  // 256 bins
+  uint32_t* sbuf = hist32 + 256;                            // short list (kShortCap keys)
   const unsigned lt_mask = (1u << lane) - 1u;
 
   for (int r = warp; r < rows; r += kWarps) {
@@ -310,8 +365,21 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
       if (n <= kk) {
         select_all = true;
       } else {
+        // every rank the row may need (k, k+1 for the gap test, 2k when the
+        // gate fires) lies in the short list when it fits
+        const int need = min(n, (a.gate ? 2 * a.top_k : a.top_k) + 1);
+        int m = 0;
+        bool short_ok = false;
+        if (need <= 32) short_ok = topk_short<1>(s, n, need, hist32, sbuf, kShortCap, &m);
+        else if (need <= 64) short_ok = topk_short<2>(s, n, need, hist32, sbuf, kShortCap, &m);
+        else if (need <= 128) short_ok = topk_short<4>(s, n, need, hist32, sbuf, kShortCap, &m);
+        // keys of the row ranked by the selection: the short list or the row
+        auto rank_key = [&](int want, int* gt, int* eq) {
+          if (short_ok) return radix_select_keys([sbuf](int q) { return sbuf[q]; }, m, want, hist32, gt, eq);
+          return radix_select(s, n, want, hist32, gt, eq);
+        };
         int n_gt, n_eq;
-        vkey = radix_select(s, n, kk - 1, hist32, &n_gt, &n_eq);
+        vkey = rank_key(kk - 1, &n_gt, &n_eq);
         take_eq = kk - n_gt;
         if (a.gate) {
           // s_(k) and s_(k+1); population std of the candidates (double)
@@ -320,12 +388,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
           if (n_gt + n_eq >= kk + 1) {
             sk1 = sk;
           } else {
-            uint32_t below = 0;
-            for (int j = lane; j < n; j += 32) {
-              const uint32_t u = fkey(s[j]);
-              if (u < vkey) below = max(below, u);
-            }
-            sk1 = key_float(warp_max_u(below));
+            int g1, e1;
+            sk1 = key_float(rank_key(kk, &g1, &e1));
           }
           double sum = 0.0;
           for (int j = lane; j < n; j += 32) sum += (double)s[j];
@@ -343,7 +407,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
             if (n <= kk) {
               select_all = true;
             } else {
-              vkey = radix_select(s, n, kk - 1, hist32, &n_gt, &n_eq);
+              vkey = rank_key(kk - 1, &n_gt, &n_eq);
               take_eq = kk - n_gt;
             }
           }
