@@ -35,7 +35,20 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention launch, from the
 # ncu capture summarised in profiles/ (None until captured for this kernel).
-NCU_ATTEND_TRAFFIC = {}
+NCU_ATTEND_TRAFFIC = {"rbs128k": 5.62e9 + 1.05e9}
+
+
+def attend_kernel_name(w) -> str:
+    """The attention kernel sbsa_attend dispatches to for workload w (the rule
+    of launch_attend in csrc/attend.cu)."""
+    big = w.dtype == "bf16" and w.block_size == 128 and w.head_dim in (64, 128)
+    pairable = big and w.group_shared and (w.n_q_heads // w.n_kv_heads) % 2 == 0
+    shape = f"{w.dtype}, B={w.block_size}, d={w.head_dim}"
+    if pairable:
+        return f"attend_pair_kernel<{w.head_dim}> (two query heads share K/V, tcgen05, {shape})"
+    if big:
+        return f"attend_ps_kernel<{w.head_dim}> (persistent, tcgen05, {shape})"
+    return f"attend_kernel (one CTA per query block, tcgen05, {shape})"
 
 
 def parse_args():
@@ -413,7 +426,7 @@ def main():
             "bound": "tensor", "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",
             "frac": att_tflops / peak_tf,
             "traffic": NCU_ATTEND_TRAFFIC.get(w.name),
-            "kernel": "attend_ps_kernel<128> (persistent, tcgen05, bf16, B=128, d=128)",
+            "kernel": attend_kernel_name(w),
             "note": f"peak = bf16_tflops burst, of {src}; achieved = 4*d*unmasked pairs / mean launch time",
         },
         "selection_roofline": {

@@ -11,7 +11,11 @@
 // stream indexed by a CTA-wide block counter g, so loads and products run
 // ahead across item boundaries.  14 warps:
 //   warp 0     TMA producer: Q of item t into Q[t % 2]; K_j, V_j of block g
-//              into a 4-stage ring (positions 2g, 2g + 1).
+//              into a 4-stage ring (positions 2g, 2g + 1).  A position is
+//              reused once the product that read it has completed, which the
+//              producer learns from the same barriers the softmax waits on
+//              (S done, PV done): each tcgen05.commit stalls the tensor pipe
+//              for about a hundred cycles, so the ring has none of its own.
 //   warp 1     TMEM owner and single-thread MMA issuer, in the order
 //              S(0), S(1), PV(0), S(2), PV(1), ...:
 //                S(g)  = Q K_j^T        -> TMEM S[g % 2]
@@ -39,7 +43,7 @@ namespace sbsa {
 namespace {
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;
-constexpr int kStages = 4;
+constexpr int kStages = 4;  // the ring release rule relies on 4 (2 blocks)
 constexpr int kThreads = 448;
 // The running maximum used for exp2 moves (and O is rescaled) only when the
 // row maximum exceeds it by more than 2^8 (P stays below 256).
@@ -57,9 +61,9 @@ struct PS {
   static constexpr int OFF_L = OFF_KV + kStages * KV_BYTES;  // row sums [item%2][half][BM]
   static constexpr int OFF_MX = OFF_L + 4 * BM * 4;          // row max [block%2][half][BM]
   static constexpr int OFF_BAR = OFF_MX + 4 * BM * 4;
-  // q_full[2] q_free[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done[2]
+  // q_full[2] q_free[2] kv_full[S] s_full[2] p_full[2] pv_done[2]
   // o_full[2] o_free[2] l_full[2] mx_ready[2][4] drain
-  static constexpr int NBARS = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 2 + 8 + 1;
+  static constexpr int NBARS = 2 + 2 + kStages + 2 + 2 + 2 + 2 + 2 + 2 + 8 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S = 0;       // S[0], S[1]: 2 x BN columns
@@ -147,8 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
   uint64_t* q_full = bar;
   uint64_t* q_free = q_full + 2;
   uint64_t* kv_full = q_free + 2;
-  uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
+  uint64_t* s_full = kv_full + kStages;
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_full = pv_done + 2;
@@ -178,10 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
       mbar_init(&l_full[b], 256);
       for (int q = 0; q < 4; ++q) mbar_init(&mx_ready[b * 4 + q], 64);
     }
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-    }
+    for (int s = 0; s < kStages; ++s) mbar_init(&kv_full[s], 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -218,6 +218,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
     int pos = 0, t = 0, q_loaded = 0;
     bool ok = true;
     Item it;
+    // Ring position q (K_b at 2b, V_b at 2b + 1) is free again once the
+    // product that read it has completed: S(b) for K_b, PV(b) for V_b.  The
+    // tensor core signals those completions anyway (to the softmax and for
+    // rescaling), so the ring needs no release commits of its own.  With 4
+    // stages, position q + 4 holds K_{b+2} or V_{b+2}, which cannot be
+    // multiplied before it is loaded, so the barrier cannot run a phase
+    // ahead of this wait.
+    auto wait_released = [&](int q) -> bool {
+      const int b = q >> 1;
+      uint64_t* bar_b = (q & 1) ? &pv_done[b & 1] : &s_full[b & 1];
+      return wait(bar_b, (b >> 1) & 1);
+    };
     for (; ok && load_item(p, t, it, lane); ++t) {
       const int qb = t & 1;
       bool good = true;
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
         for (int half = 0; half < 2; ++half) {
           const int st = pos % kStages;
           if (lane == 0) {
-            good = wait(&kv_empty[st], ((pos / kStages) & 1) ^ 1);
+            good = pos < kStages || wait_released(pos - kStages);
             if (good) {
               mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
               const CUtensorMap* m = half ? &p.tm_v : &p.tm_k;
@@ -274,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
       } else {
         // wait for the MMA thread's last asynchronous releases
         for (int q = first; q < pos; ++q)
-          if (!wait(&kv_empty[q % kStages], (q / kStages) & 1)) break;
+          if (!wait_released(q)) break;
         for (int u = (q_loaded >= 2 ? q_loaded - 2 : 0); u < q_loaded; ++u)
           if (!wait(&q_free[u & 1], (u >> 1) & 1)) break;
       }
@@ -283,6 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
     // ================================================================ MMA
     const uint32_t q_base = smem_u32(sQ);
     const uint32_t kv_base = smem_u32(sKV);
+    // start-address-0 descriptors of the Q and K tiles (K-major, 128-byte
+    // swizzle) and of V (MN-major); stage and step offsets are added to the
+    // start address field
+    const uint64_t q_desc0 = smem_desc(q_base, 16, 1024);
+    const uint64_t k_desc0 = smem_desc(kv_base, 16, 1024);
+    const uint64_t v_desc0 = smem_desc(kv_base, BN * 128, 1024);
     struct Pending {
       int g, t, b, last;  // block counter, item, block within item, last of item
     };
@@ -297,15 +315,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
       const int st = vpos % kStages;
       if (!wait(&kv_full[st], (vpos / kStages) & 1)) return false;
       tc_fence_after();
-      const uint32_t v_base = kv_base + st * C::KV_BYTES;
+      // descriptors of the 8 K-steps differ only in the start address
+      // field (16 rows of 128 bytes = 128 in units of 16 bytes per step)
+      const uint64_t bd0 = v_desc0 + (uint64_t)(st * (C::KV_BYTES >> 4));
       const uint32_t a_col = tmem + C::TM_S + (pv.g & 1) * BN;
       const uint32_t o_col = tmem + C::TM_O + (pv.t & 1) * D;
+      const uint32_t acc0 = pv.b > 0 ? 1u : 0u;
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk) {
-        const uint64_t bd = smem_desc(v_base + kk * 16 * 128, BN * 128, 1024);
-        umma_f16_ts(o_col, a_col + kk * 8, bd, C::IDESC_O, (pv.b > 0 || kk > 0) ? 1u : 0u);
-      }
-      umma_commit(&kv_empty[st]);
+      for (int kk = 0; kk < BN / 16; ++kk)
+        umma_f16_ts(o_col, a_col + kk * 8, bd0 + (uint64_t)(kk * 128), C::IDESC_O, kk > 0 ? 1u : acc0);
       umma_commit(&pv_done[pv.g & 1]);
       if (pv.last) umma_commit(&o_full[pv.t & 1]);
       return true;
@@ -342,17 +360,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
           good = wait(&kv_full[st], (kpos / kStages) & 1);
           if (good) {
             tc_fence_after();
-            const uint32_t qa = q_base + qb * C::Q_BYTES;
-            const uint32_t ka = kv_base + st * C::KV_BYTES;
+            const uint64_t ad0 = q_desc0 + (uint64_t)(qb * (C::Q_BYTES >> 4));
+            const uint64_t bd0 = k_desc0 + (uint64_t)(st * (C::KV_BYTES >> 4));
             const uint32_t s_col = tmem + C::TM_S + (g & 1) * BN;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
+              // 32 bytes per K-step inside a 128-byte swizzle atom, then the
+              // next atom (BM or BN rows of 128 bytes) every 4 steps
               const int kb = kk * 32;
-              const uint64_t ad = smem_desc(qa + (kb / 128) * (BM * 128) + (kb % 128), 16, 1024);
-              const uint64_t bd = smem_desc(ka + (kb / 128) * (BN * 128) + (kb % 128), 16, 1024);
-              umma_f16_ss(s_col, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+              const uint64_t da = (uint64_t)(((kb / 128) * (BM * 128) + (kb % 128)) >> 4);
+              const uint64_t db = (uint64_t)(((kb / 128) * (BN * 128) + (kb % 128)) >> 4);
+              umma_f16_ss(s_col, ad0 + da, bd0 + db, C::IDESC_S, kk > 0 ? 1u : 0u);
             }
-            umma_commit(&kv_empty[st]);
             umma_commit(&s_full[g & 1]);
             if (last) umma_commit(&q_free[qb]);
             if (have_prev) good = issue_pv(prev);
