@@ -38,6 +38,43 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 NCU_ATTEND_TRAFFIC = {"rbs128k": 5.62e9 + 1.05e9}
 
 
+def selection_stats(w, p, st, meta) -> dict:
+    """What the selection produced: rows whose gap gate fired, rows the
+    radius rescue added blocks to, planted needles found, and the attention
+    stage's algorithmic bytes (Q + O + each distinct K/V block once)."""
+    import torch
+    from block_sparse_attention_sbsa_b200 import sbsa
+    flags = st.flags.to(torch.int32)
+    out = {
+        "rows": int(flags.numel()),
+        "gate_fired_fraction": float(((flags & sbsa.FLAG_GATE) != 0).float().mean()),
+        "rescued_rows_fraction": float(((flags & sbsa.FLAG_RESCUE) != 0).float().mean()),
+    }
+    nb, kmax = w.n_blocks, st.idx.shape[-1]
+    valid = torch.arange(kmax, device=st.idx.device).view(1, 1, -1) < st.cnt.unsqueeze(-1)
+    ids = torch.where(valid, st.idx, torch.full_like(st.idx, -1)).to(torch.int64)
+    # distinct (kv head, key block) pairs named by any list
+    grp = 1 if w.group_shared else w.n_q_heads // w.n_kv_heads
+    kvh = (torch.arange(ids.shape[0], device=ids.device) // grp).view(-1, 1, 1).expand_as(ids)
+    used = torch.zeros(w.n_kv_heads * nb, dtype=torch.bool, device=ids.device)
+    sel = ids >= 0
+    used[(kvh[sel] * nb + ids[sel]).unique()] = True
+    es = 2 if w.dtype == "bf16" else 4
+    blk = w.block_size * w.head_dim * es
+    out["distinct_kv_blocks"] = int(used.sum())
+    out["attend_algorithmic_bytes"] = int(2 * w.n_q_heads * w.seq_len * w.head_dim * es
+                                          + 2 * int(used.sum()) * blk)
+    needles = meta.get("needles", [])
+    if needles and w.group_shared:
+        hits = 0
+        idx_cpu, cnt_cpu = st.idx.cpu(), st.cnt.cpu()
+        for (g, pos, qb) in needles:
+            row = idx_cpu[g, qb, :int(cnt_cpu[g, qb])]
+            hits += int((row == pos // w.block_size).any())
+        out["needle_hit_rate"] = hits / len(needles)
+    return out
+
+
 def attend_kernel_name(w) -> str:
     """The attention kernel sbsa_attend dispatches to for workload w (the rule
     of launch_attend in csrc/attend.cu)."""
@@ -337,6 +374,7 @@ def main():
     pairs = sbsa.attended_pairs(p, st.cnt)
     attend_flops = 4.0 * w.head_dim * pairs
     mean_cnt = float(st.cnt.float().mean())
+    sel_stats = selection_stats(w, p, st, data.get("meta", {}))
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -436,6 +474,13 @@ def main():
         },
         "stages_ms": {"pool": pool_ms, "select": sel_ms, "attend": att_ms},
         "selected_blocks_per_row": mean_cnt,
+        "selection_stats": sel_stats,
+        "attend_bytes": {
+            "algorithmic": sel_stats["attend_algorithmic_bytes"],
+            "gbs": sel_stats["attend_algorithmic_bytes"] / (att_ms / 1000.0) / 1e9,
+            "note": "Q + O + every distinct (kv head, block) of K and V a list names, once each; "
+                    "far below the HBM peak: attention is not bound by DRAM",
+        },
         "attended_pairs": pairs,
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
