@@ -26,6 +26,10 @@ Sources (web pages; cited by title and section):
 * "MiniMax presenta MSA ..." (iaonda.com), section "Que es MSA y como
   funciona?": one top-k block selection per GQA group by a light index
   branch, full attention over the selected blocks only.
+* The uncertainty-gated page, Metodologia step 1 and Contribuciones
+  (Componibilidad): the block-scoring backbone is interchangeable; besides
+  SSA-style mean pooling it names Quest's per-coordinate upper bounds from
+  the block's K-min / K-max.
 
 Readings where the pages are silent (each one also listed in the design
 notes): the radius is the largest l2 distance of a block's keys from its
@@ -37,6 +41,8 @@ the k-th minus (k+1)-th largest score is below margin * (population std of
 the row's candidate scores); cumulative mass uses a softmax over the
 candidates and keeps the shortest prefix of the ranked order whose mass
 reaches the threshold; the rescue test is (q.c + |q| r) * scale > tau.
+The K-min/K-max backbone bounds q.k over the block's keys coordinate by
+coordinate: sum_d max(q_d * min_d, q_d * max_d), scaled like the mean score.
 """
 from __future__ import annotations
 
@@ -94,6 +100,23 @@ def pool_keys(k, block: int, with_radius: bool = True, heads=None):
     return c, (r if with_radius else None)
 
 
+def pool_keys_minmax(k, block: int):
+    """Per-coordinate minimum and maximum of the keys of each block (the
+    K-min / K-max table of the upper-bound backbone).  Returns (kmin, kmax),
+    each [Hkv, NB, d]."""
+    hk, n, d = k.shape
+    nb = n_blocks(n, block)
+    kmin = np.zeros((hk, nb, d))
+    kmax = np.zeros((hk, nb, d))
+    for g in range(hk):
+        kg = _f64(k[g])
+        for j in range(nb):
+            rows = kg[j * block:min(n, (j + 1) * block)]
+            kmin[g, j] = rows.min(axis=0)
+            kmax[g, j] = rows.max(axis=0)
+    return kmin, kmax
+
+
 def pool_queries(q, block: int, group: int = 1, blocks=None):
     """Pooled query of block i: the mean of the block's query rows (one query
     tile per block).  With ``group`` > 1 (one selection per GQA group), the
@@ -123,6 +146,15 @@ def block_scores(qbar_i, c_g, i: int, scale: float):
     float32 (the precision the selection decision is taken in)."""
     s = (c_g[:i] @ qbar_i) * scale
     return s.astype(np.float32)
+
+
+def block_bounds_minmax(qbar_i, kmin_g, kmax_g, i: int, scale: float):
+    """Upper-bound backbone: s_j = sum_d max(qbar_d * min_jd, qbar_d * max_jd)
+    * scale for the candidates j < i -- the largest q.k over any key inside
+    the block's coordinate box -- rounded to float32."""
+    lo = kmin_g[:i] * qbar_i
+    hi = kmax_g[:i] * qbar_i
+    return (np.maximum(lo, hi).sum(axis=1) * scale).astype(np.float32)
 
 
 def rescue_bounds(qbar_i, c_g, r_g, i: int, scale: float):
@@ -209,7 +241,7 @@ def select_row(s, i: int, *, mode: str, top_k_: int = 0, mass: float = 0.0,
 
 def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
            mass: float = 0.0, margin=None, tau=None, scale: float,
-           kv_of_sel=None, max_blocks: int, rows=None):
+           kv_of_sel=None, max_blocks: int, rows=None, minmax=None):
     """Lists for every selection head hs and query block i (or the (hs, i)
     pairs in ``rows``).  ``qbar`` is [Hs, NB, d_s] and ``c``/``r`` are the key
     tables [Hkv, NB, ...]; ``kv_of_sel(hs)`` gives the kv head whose key table
@@ -223,7 +255,10 @@ def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
     pairs = rows if rows is not None else [(h, i) for h in range(hs_n) for i in range(nb)]
     for (h, i) in pairs:
         g = kv_of_sel(h)
-        s = block_scores(qbar[h, i], c[g], i, scale)
+        if minmax is None:
+            s = block_scores(qbar[h, i], c[g], i, scale)
+        else:
+            s = block_bounds_minmax(qbar[h, i], minmax[0][g], minmax[1][g], i, scale)
         ub = rescue_bounds(qbar[h, i], c[g], r[g], i, scale) if tau is not None else None
         ids, fl = select_row(s, i, mode=mode, top_k_=top_k_, mass=mass,
                              margin=margin, ub=ub, tau=tau)
@@ -324,7 +359,7 @@ def attend_dense_masked(q, k, v, idx, cnt, *, block: int, scale: float,
 def prefill(q, k, v, *, block: int, mode: str, top_k_: int = 0,
             mass: float = 0.0, margin=None, tau=None, group_shared: bool = False,
             q_idx=None, k_idx=None, max_blocks: int, scale=None,
-            score_scale=None, sel_rows=None, attend_rows=None):
+            score_scale=None, sel_rows=None, attend_rows=None, backbone: str = "mean"):
     """Selection tables and lists from the index tensors (q_idx/k_idx when
     given, else q/k), then attention over the lists.  ``sel_rows`` restricts
     selection to (hs, i) pairs, ``attend_rows`` restricts attention to
@@ -341,6 +376,14 @@ def prefill(q, k, v, *, block: int, mode: str, top_k_: int = 0,
     c, r = pool_keys(ks, block, with_radius=tau is not None)
     if r is None:
         r = np.zeros(c.shape[:2])
+    if backbone == "minmax":
+        if tau is not None:
+            raise ValueError("the rescue branch needs the mean backbone")
+        minmax = pool_keys_minmax(ks, block)
+    elif backbone == "mean":
+        minmax = None
+    else:
+        raise ValueError(backbone)
     if group_shared:
         qbar = pool_queries(qs, block, group=grp)
         kv_of_sel = lambda hs: hs
@@ -350,7 +393,8 @@ def prefill(q, k, v, *, block: int, mode: str, top_k_: int = 0,
     idx, cnt, flags = select(qbar, c, r, block_count=nb, mode=mode, top_k_=top_k_,
                              mass=mass, margin=margin, tau=tau, scale=score_scale,
                              kv_of_sel=kv_of_sel, max_blocks=max_blocks,
-                             rows=sel_rows)
+                             rows=sel_rows, minmax=minmax)
     out = attend(q, k, v, idx, cnt, block=block, scale=scale,
                  group_shared=group_shared, rows=attend_rows)
-    return dict(c=c, r=r, qbar=qbar, idx=idx, cnt=cnt, flags=flags, o=out)
+    return dict(c=c, r=r, qbar=qbar, idx=idx, cnt=cnt, flags=flags, o=out,
+                minmax=minmax)

@@ -361,3 +361,87 @@ def test_rbs_rescue_adds_the_past_outlier_blocks():
             assert past <= ids
     # the base branch stays sparse: on average a handful of blocks per row
     assert res["cnt"].mean() < 16
+
+
+# --------------------------------------------------------------------------
+# K-min / K-max upper-bound backbone (uncertainty-gated page, Metodologia
+# step 1 and Componibilidad: per-coordinate bounds from K-min / K-max)
+# --------------------------------------------------------------------------
+
+def test_minmax_table_is_the_tightest_box_around_each_block():
+    rng = np.random.default_rng(21)
+    k = rng.standard_normal((2, 203, 8)).astype(np.float32)  # ragged last block
+    kmin, kmax = O.pool_keys_minmax(k, 64)
+    for g in range(2):
+        for j in range(O.n_blocks(203, 64)):
+            rows = k[g, j * 64:min(203, (j + 1) * 64)].astype(np.float64)
+            # every key inside the box ...
+            assert (rows >= kmin[g, j] - 0).all() and (rows <= kmax[g, j] + 0).all()
+            # ... and every face touched by some key
+            for c in range(8):
+                assert (rows[:, c] == kmin[g, j, c]).any()
+                assert (rows[:, c] == kmax[g, j, c]).any()
+
+
+def test_minmax_bound_is_the_maximum_over_the_box_corners():
+    """q.x over the box [lo, hi] is linear, so its maximum sits at a corner:
+    brute force over all 2^d corners must give the same value."""
+    import itertools
+    rng = np.random.default_rng(22)
+    d = 5
+    for trial in range(20):
+        lo = rng.standard_normal((3, d))
+        hi = lo + rng.random((3, d)) * 2
+        q = rng.standard_normal(d)
+        got = O.block_bounds_minmax(q, lo, hi, 3, 1.0).astype(np.float64)
+        for j in range(3):
+            best = max(float(np.dot(q, np.where(np.array(corner), hi[j], lo[j])))
+                       for corner in itertools.product([0, 1], repeat=d))
+            assert got[j] == pytest.approx(best, rel=1e-6, abs=1e-6)
+
+
+def test_minmax_bound_dominates_every_key_and_is_exact_for_a_point_block():
+    rng = np.random.default_rng(23)
+    k = rng.standard_normal((1, 256, 16))
+    k[0, 128:192] = k[0, 128]  # block 2: one key repeated
+    kmin, kmax = O.pool_keys_minmax(k, 64)
+    q = rng.standard_normal(16)
+    ub = O.block_bounds_minmax(q, kmin[0], kmax[0], 4, 1.0).astype(np.float64)
+    for j in range(4):
+        dots = k[0, j * 64:(j + 1) * 64] @ q
+        assert ub[j] >= dots.max() - 1e-5
+    assert ub[2] == pytest.approx(float(k[0, 128] @ q), rel=1e-6)
+    # sign-definite queries pick one face: q >= 0 -> q.max, q <= 0 -> q.min
+    qp = np.abs(q)
+    assert O.block_bounds_minmax(qp, kmin[0], kmax[0], 4, 1.0) == pytest.approx(
+        (kmax[0] @ qp).astype(np.float32), rel=1e-6)
+    assert O.block_bounds_minmax(-qp, kmin[0], kmax[0], 4, 1.0) == pytest.approx(
+        (kmin[0] @ -qp).astype(np.float32), rel=1e-6)
+
+
+def test_minmax_backbone_finds_the_spread_out_block_the_mean_misses():
+    """A block whose keys swing to +-10 along the query direction has a mean
+    near 0 (invisible to the centroid score) but the largest bound."""
+    rng = np.random.default_rng(24)
+    n, b, d = 8 * 32, 32, 16
+    q = rng.standard_normal((1, n, d)) * 0.1
+    k = rng.standard_normal((1, n, d)) * 0.1
+    v = rng.standard_normal((1, n, d))
+    u = np.zeros(d)
+    u[0] = 1.0
+    q[0, 7 * b:] += 2.0 * u                     # the last query block looks along e_0
+    k[0, 3 * b:4 * b:2, 0] += 10.0              # block 3: alternate keys at +10 ...
+    k[0, 3 * b + 1:4 * b:2, 0] -= 10.0          # ... and -10 (mean unchanged)
+    k[0, 5 * b:6 * b, 0] += 0.5                 # block 5: a modest shift of the mean
+    common = dict(block=b, mode="topk", top_k_=1, max_blocks=2)
+    mean = O.prefill(q, k, v, backbone="mean", **common)
+    mm = O.prefill(q, k, v, backbone="minmax", **common)
+    assert mean["idx"][0, 7, :2].tolist() == [5, 7]
+    assert mm["idx"][0, 7, :2].tolist() == [3, 7]
+
+
+def test_minmax_backbone_rejects_the_rescue_branch():
+    x = np.zeros((1, 64, 8))
+    with pytest.raises(ValueError):
+        O.prefill(x, x, x, block=32, mode="cummass", mass=0.9, tau=1.0, max_blocks=2,
+                  backbone="minmax")
