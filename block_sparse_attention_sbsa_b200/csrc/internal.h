@@ -13,8 +13,9 @@ struct PoolJob {
   const void* x;
   int n_heads;
   int group;
-  float* cent;
+  float* cent;  // [n_heads/group, NB, dim] means, or nullptr when mm is set
   float* rad;
+  float* mm;    // [n_heads, NB, 2, dim] coordinate-wise min then max, or nullptr
 };
 
 // Launch pooling of up to two jobs (same dtype and dim) as one grid.
@@ -23,7 +24,7 @@ cudaError_t launch_pool(int dtype, int dim, int seq_len, int block, const PoolJo
 
 struct SelectArgs {
   const float* qc;   // [Hs, NB, ds]
-  const float* kc;   // [Hkv, NB, ds]
+  const float* kc;   // [Hkv, NB, ds] centroids, or [Hkv, NB, 2, ds] min/max (minmax)
   const float* kr;   // [Hkv, NB] or nullptr
   int32_t* idx;      // [Hs, NB, kmax]
   int32_t* cnt;      // [Hs, NB]
@@ -34,6 +35,7 @@ struct SelectArgs {
   int ds;
   int kmax;
   int mode;          // SBSA_TOPK | SBSA_CUMMASS
+  int minmax;        // 1: upper-bound scores from the min/max table
   int top_k;
   float mass;
   int gate;

@@ -1,6 +1,7 @@
 // Block pooling: centroid (mean of a block's rows) and radius (largest l2
 // distance of a row from the centroid), optionally averaged over a group of
-// consecutive heads.
+// consecutive heads; or the coordinate-wise minimum and maximum of a block's
+// rows (the K-min / K-max table of the upper-bound scoring backbone).
 //
 // "RBS-Attention" (iaonda.com), method paragraph: key blocks are summarised
 // by a centroid and a dynamic, prompt/layer/head-dependent key-block radius.
@@ -87,6 +88,45 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
   const int vec = tid % VPR;
   const int rsub = tid / VPR;
   const bool want_r = job.rad != nullptr;
+
+  if (job.mm) {
+    // coordinate-wise minimum and maximum over the block's rows
+    float mn[E], mx[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      mn[e] = INFINITY;
+      mx[e] = -INFINITY;
+    }
+    const T* base = static_cast<const T*>(job.x) + ((size_t)hs * g.n + row0) * DIM + vec * E;
+    for (int r = rsub; r < nrows; r += RPP) {
+      float f[E];
+      Vec16<T>::to_float(ld_stream(base + (size_t)r * DIM), f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        mn[e] = fminf(mn[e], f[e]);
+        mx[e] = fmaxf(mx[e], f[e]);
+      }
+    }
+    float* out = job.mm + ((size_t)hs * g.nb + j) * 2 * DIM;
+#pragma unroll
+    for (int e = 0; e < E; ++e) red[rsub][vec * E + e] = mn[e];
+    __syncthreads();
+    for (int col = tid; col < DIM; col += kPoolThreads) {
+      float m = red[0][col];
+      for (int r = 1; r < RPP; ++r) m = fminf(m, red[r][col]);
+      out[col] = m;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < E; ++e) red[rsub][vec * E + e] = mx[e];
+    __syncthreads();
+    for (int col = tid; col < DIM; col += kPoolThreads) {
+      float m = red[0][col];
+      for (int r = 1; r < RPP; ++r) m = fmaxf(m, red[r][col]);
+      out[DIM + col] = m;
+    }
+    return;
+  }
 
   float acc[E];
 #pragma unroll

@@ -62,6 +62,9 @@ int validate(const sbsa_params* p, Derived* d) {
   if (p->gate && !(p->gate_margin >= 0.f && std::isfinite(p->gate_margin)))
     return SBSA_ERR_INVALID_ARG;
   if (p->rescue && std::isnan(p->rescue_tau)) return SBSA_ERR_INVALID_ARG;
+  if (p->backbone != SBSA_BACKBONE_MEAN && p->backbone != SBSA_BACKBONE_MINMAX)
+    return SBSA_ERR_INVALID_ARG;
+  if (p->backbone == SBSA_BACKBONE_MINMAX && p->rescue) return SBSA_ERR_INVALID_ARG;
   if (!(p->sm_scale >= 0.f) || !std::isfinite(p->sm_scale)) return SBSA_ERR_INVALID_ARG;
   if (!(p->score_scale >= 0.f) || !std::isfinite(p->score_scale)) return SBSA_ERR_INVALID_ARG;
   Derived o;
@@ -100,7 +103,8 @@ WsLayout layout(const sbsa_params* p, const Derived& d, bool lists) {
   w.qc = off;
   off = round_up(off + (size_t)d.hs * d.nb * d.ds * 4, 256);
   w.kc = off;
-  off = round_up(off + (size_t)p->n_kv_heads * d.nb * d.ds * 4, 256);
+  const size_t tables_per_block = p->backbone == SBSA_BACKBONE_MINMAX ? 2 : 1;
+  off = round_up(off + tables_per_block * p->n_kv_heads * d.nb * d.ds * 4, 256);
   w.kr = off;
   off = round_up(off + (p->rescue ? (size_t)p->n_kv_heads * d.nb * 4 : 0), 256);
   w.idx = off;
@@ -130,6 +134,7 @@ SelectArgs select_args(const sbsa_params* p, const Derived& d, const float* qc, 
   a.ds = d.ds;
   a.kmax = p->max_blocks;
   a.mode = p->select_mode;
+  a.minmax = p->backbone == SBSA_BACKBONE_MINMAX ? 1 : 0;
   a.top_k = p->top_k;
   a.mass = p->mass_threshold;
   a.gate = p->gate ? 1 : 0;
@@ -170,7 +175,7 @@ using namespace sbsa;
 
 extern "C" {
 
-int sbsa_version(void) { return 100; }
+int sbsa_version(void) { return 101; }
 
 const char* sbsa_status_string(int code) {
   switch (code) {
@@ -195,7 +200,21 @@ int sbsa_pool_blocks(const sbsa_params* p, const void* x, int n_heads, int dim, 
   if (dim != 64 && dim != 128) return SBSA_ERR_UNSUPPORTED;
   if (radii && group != 1) return SBSA_ERR_INVALID_ARG;
   if (!aligned16(x)) return SBSA_ERR_INVALID_ARG;
-  PoolJob job{x, n_heads, group, centroids, radii};
+  PoolJob job{x, n_heads, group, centroids, radii, nullptr};
+  return cuda_code(launch_pool(p->dtype, dim, p->seq_len, p->block_size, &job, 1,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+int sbsa_pool_minmax(const sbsa_params* p, const void* x, int n_heads, int dim, float* minmax,
+                     void* stream) {
+  if (!p || !x || !minmax) return SBSA_ERR_INVALID_ARG;
+  if (p->seq_len < 1 || p->block_size <= 0) return SBSA_ERR_INVALID_ARG;
+  if (p->dtype != SBSA_BF16 && p->dtype != SBSA_FP32) return SBSA_ERR_INVALID_ARG;
+  if (p->block_size != 64 && p->block_size != 128) return SBSA_ERR_UNSUPPORTED;
+  if (n_heads < 1) return SBSA_ERR_INVALID_ARG;
+  if (dim != 64 && dim != 128) return SBSA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(minmax)) return SBSA_ERR_INVALID_ARG;
+  PoolJob job{x, n_heads, 1, nullptr, nullptr, minmax};
   return cuda_code(launch_pool(p->dtype, dim, p->seq_len, p->block_size, &job, 1,
                                static_cast<cudaStream_t>(stream)));
 }
@@ -262,9 +281,10 @@ int sbsa_prefill(const sbsa_params* p, const void* q, const void* k, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const void* xs_k = p->index_dim ? k_idx : k;
   const void* xs_q = p->index_dim ? q_idx : q;
+  const bool minmax = p->backbone == SBSA_BACKBONE_MINMAX;
   PoolJob jobs[2] = {
-      {xs_k, p->n_kv_heads, 1, kc, kr},
-      {xs_q, p->n_q_heads, p->group_shared ? d.group : 1, qc, nullptr},
+      {xs_k, p->n_kv_heads, 1, minmax ? nullptr : kc, kr, minmax ? kc : nullptr},
+      {xs_q, p->n_q_heads, p->group_shared ? d.group : 1, qc, nullptr, nullptr},
   };
   rc = cuda_code(launch_pool(p->dtype, d.ds, p->seq_len, p->block_size, jobs, 2, s));
   if (rc) return rc;

@@ -12,6 +12,11 @@
 // rescue branch through the block radius, each with its own threshold, masks
 // united.  "MiniMax presenta MSA": one selection per GQA group.
 //
+// Scores come from the centroids (mean backbone) or, with the K-min / K-max
+// backbone ("Uncertainty-gated selection", Metodologia step 1 and
+// Componibilidad: Quest-style per-coordinate upper bounds), from
+// sum_d max(q_d min_d, q_d max_d) over the block's coordinate box.
+//
 // Layout of one CTA: R (up to 16) consecutive query blocks of one selection
 // head.  Phase 1 computes their scores against every earlier key block into
 // shared memory: each thread streams whole key-centroid rows from L2 in
@@ -75,12 +80,6 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
 // block id (ids are complemented so that a larger composite ranks first).
 __device__ __forceinline__ uint64_t rank_key(float s, int j) {
   return ((uint64_t)fkey(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
-}
-
-__device__ __forceinline__ uint32_t warp_max_u(uint32_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
 }
 
 // Key of descending rank `want` (0-based) among key(0..n).  *n_gt gets the
@@ -317,8 +316,35 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
   // and streams their centroid rows (fp32) from L2 in 16-byte pieces, dotting
   // each piece with the R pooled queries read from shared memory (every lane
   // reads the same address: one broadcast per row).
+  if (a.minmax) {
+    // Upper-bound backbone: s_j = sum_d max(q_d min_jd, q_d max_jd), the two
+    // table rows of block j streamed like a centroid row.
+    const float* km = a.kc + (size_t)g * a.nb * 2 * DS;
+    for (int j = tid; j < jend; j += kSelThreads) {
+      const float4* lo = reinterpret_cast<const float4*>(km + (size_t)j * 2 * DS);
+      const float4* hi = lo + DS / 4;
+      float acc[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[r] = 0.f;
+#pragma unroll 2
+      for (int k4 = 0; k4 < DS / 4; ++k4) {
+        const float4 l4 = __ldg(lo + k4);
+        const float4 h4 = __ldg(hi + k4);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const float4 q4 = *reinterpret_cast<const float4*>(qs + r * DS + 4 * k4);
+          acc[r] += fmaxf(q4.x * l4.x, q4.x * h4.x);
+          acc[r] += fmaxf(q4.y * l4.y, q4.y * h4.y);
+          acc[r] += fmaxf(q4.z * l4.z, q4.z * h4.z);
+          acc[r] += fmaxf(q4.w * l4.w, q4.w * h4.w);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) sc[r * score_stride + j] = acc[r] * a.score_scale;
+    }
+  }
   const float* kc = a.kc + (size_t)g * a.nb * DS;
-  for (int j = tid; j < jend; j += kSelThreads) {
+  for (int j = a.minmax ? jend : tid; j < jend; j += kSelThreads) {
     const float4* crow = reinterpret_cast<const float4*>(kc + (size_t)j * DS);
     float acc[R];
 #pragma unroll

@@ -21,9 +21,10 @@ LIB_PATH = os.path.join(_HERE, "libsbsa.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
 BF16, FP32 = 0, 1
 TOPK, CUMMASS = 0, 1
+BACKBONE_MEAN, BACKBONE_MINMAX = 0, 1
 FLAG_GATE, FLAG_RESCUE = 1, 2
 
-SYMBOLS = ["sbsa_pool_blocks", "sbsa_select", "sbsa_attend", "sbsa_prefill",
+SYMBOLS = ["sbsa_pool_blocks", "sbsa_pool_minmax", "sbsa_select", "sbsa_attend", "sbsa_prefill",
            "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string",
            "sbsa_version", "sbsa_debug_wait_timeout"]
 
@@ -54,6 +55,7 @@ class Params(ctypes.Structure):
         ("max_blocks", ctypes.c_int),
         ("sm_scale", ctypes.c_float),
         ("score_scale", ctypes.c_float),
+        ("backbone", ctypes.c_int),
     ]
 
     @property
@@ -79,6 +81,7 @@ def _load() -> ctypes.CDLL:
     vp, i32p, f32p, u8p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
     ci = ctypes.c_int
     lib.sbsa_pool_blocks.argtypes = [P, vp, ci, ci, ci, f32p, f32p, vp]
+    lib.sbsa_pool_minmax.argtypes = [P, vp, ci, ci, f32p, vp]
     lib.sbsa_select.argtypes = [P, f32p, f32p, f32p, i32p, i32p, u8p, vp]
     lib.sbsa_attend.argtypes = [P, vp, vp, vp, i32p, i32p, vp, vp]
     lib.sbsa_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i32p, i32p, u8p, vp]
@@ -133,7 +136,7 @@ def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
 def make_params(*, n_q_heads, n_kv_heads, seq_len, head_dim, block_size, dtype="bf16",
                 select_mode="topk", top_k=0, mass_threshold=0.0, rescue_tau=None,
                 gate_margin=None, group_shared=False, index_dim=0, max_blocks=None,
-                sm_scale=0.0, score_scale=0.0) -> Params:
+                sm_scale=0.0, score_scale=0.0, backbone="mean") -> Params:
     p = Params()
     p.n_q_heads, p.n_kv_heads, p.seq_len = n_q_heads, n_kv_heads, seq_len
     p.head_dim, p.block_size = head_dim, block_size
@@ -157,6 +160,8 @@ def make_params(*, n_q_heads, n_kv_heads, seq_len, head_dim, block_size, dtype="
     p.max_blocks = max_blocks
     p.sm_scale = sm_scale
     p.score_scale = score_scale
+    p.backbone = ({"mean": BACKBONE_MEAN, "minmax": BACKBONE_MINMAX}[backbone]
+                  if isinstance(backbone, str) else int(backbone))
     return p
 
 
@@ -167,7 +172,8 @@ def params_for(w) -> Params:
                        select_mode=w.select_mode, top_k=w.top_k,
                        mass_threshold=w.mass_threshold, rescue_tau=w.rescue_tau,
                        gate_margin=w.gate_margin, group_shared=w.group_shared,
-                       index_dim=w.index_dim, max_blocks=w.max_blocks)
+                       index_dim=w.index_dim, max_blocks=w.max_blocks,
+                       backbone=getattr(w, "backbone", "mean"))
 
 
 _TORCH_DT = {BF16: torch.bfloat16, FP32: torch.float32}
@@ -187,12 +193,28 @@ def pool_blocks(p: Params, x: torch.Tensor, group: int = 1, radius: bool = False
     return cent, rad
 
 
+def pool_minmax(p: Params, x: torch.Tensor, stream=None):
+    """Coordinate-wise minimum and maximum of each block of x [H, N, dim]:
+    a [H, NB, 2, dim] table (minima, then maxima)."""
+    _need(x, "x", _TORCH_DT[p.dtype])
+    h, n, dim = x.shape
+    if n != p.seq_len:
+        raise ValueError("x.shape[1] must equal seq_len")
+    mm = torch.empty(h, p.n_blocks, 2, dim, device=x.device, dtype=torch.float32)
+    _check(lib.sbsa_pool_minmax(ctypes.byref(p), _ptr(x), h, dim, _ptr(mm), _stream(stream)),
+           "sbsa_pool_minmax")
+    return mm
+
+
 def select(p: Params, q_cent: torch.Tensor, k_cent: torch.Tensor,
            k_radius: Optional[torch.Tensor] = None, stream=None, with_flags: bool = True):
-    """Block lists (idx [Hs, NB, Kmax], cnt [Hs, NB], flags [Hs, NB])."""
+    """Block lists (idx [Hs, NB, Kmax], cnt [Hs, NB], flags [Hs, NB]).  k_cent
+    is the centroid table [Hkv, NB, ds], or the min/max table [Hkv, NB, 2, ds]
+    of pool_minmax when p.backbone is BACKBONE_MINMAX."""
     nb, hs, ds = p.n_blocks, p.n_sel_heads, p.score_dim
     _need(q_cent, "q_cent", torch.float32, (hs, nb, ds))
-    _need(k_cent, "k_cent", torch.float32, (p.n_kv_heads, nb, ds))
+    kshape = (p.n_kv_heads, nb, 2, ds) if p.backbone == BACKBONE_MINMAX else (p.n_kv_heads, nb, ds)
+    _need(k_cent, "k_cent", torch.float32, kshape)
     if p.rescue:
         _need(k_radius, "k_radius", torch.float32, (p.n_kv_heads, nb))
     dev = q_cent.device
@@ -284,15 +306,17 @@ def get_status(stream=None) -> int:
 
 class Staged:
     """The prefill as its separate C-ABI stages on preallocated buffers:
-    pool keys (+ radii), pool queries, select, attend.  Each method is one
-    library call and allocates nothing; the kernels are the ones
-    sbsa_prefill launches (which merges the two pooling jobs into one grid)."""
+    pool keys (centroids + radii, or the min/max table of the upper-bound
+    backbone), pool queries, select, attend.  Each method is one library call
+    and allocates nothing; the kernels are the ones sbsa_prefill launches
+    (which merges the two pooling jobs into one grid)."""
 
     def __init__(self, p: Params, device="cuda"):
         self.p = p
         nb, hs, ds, hk = p.n_blocks, p.n_sel_heads, p.score_dim, p.n_kv_heads
         f32 = dict(device=device, dtype=torch.float32)
-        self.kc = torch.empty(hk, nb, ds, **f32)
+        self.minmax = p.backbone == BACKBONE_MINMAX
+        self.kc = torch.empty((hk, nb, 2, ds) if self.minmax else (hk, nb, ds), **f32)
         self.kr = torch.empty(hk, nb, **f32) if p.rescue else None
         self.qc = torch.empty(hs, nb, ds, **f32)
         self.idx = torch.empty(hs, nb, p.max_blocks, device=device, dtype=torch.int32)
@@ -304,8 +328,12 @@ class Staged:
         p, s = self.p, _stream(stream)
         ds = p.score_dim
         grp = (p.n_q_heads // p.n_kv_heads) if p.group_shared else 1
-        _check(lib.sbsa_pool_blocks(self._p, _ptr(k_src), p.n_kv_heads, ds, 1, _ptr(self.kc),
-                                    _ptr(self.kr), s), "sbsa_pool_blocks")
+        if self.minmax:
+            _check(lib.sbsa_pool_minmax(self._p, _ptr(k_src), p.n_kv_heads, ds, _ptr(self.kc), s),
+                   "sbsa_pool_minmax")
+        else:
+            _check(lib.sbsa_pool_blocks(self._p, _ptr(k_src), p.n_kv_heads, ds, 1, _ptr(self.kc),
+                                        _ptr(self.kr), s), "sbsa_pool_blocks")
         _check(lib.sbsa_pool_blocks(self._p, _ptr(q_src), p.n_q_heads, ds, grp, _ptr(self.qc),
                                     None, s), "sbsa_pool_blocks")
 

@@ -25,6 +25,9 @@ Five workload families, one per configuration of the benchmark suite:
 * ``msa512k`` 64/8 heads, d=128, N=524288, B=128, bf16, top-32 shared per GQA
               group on index tensors of width 64 (Q_idx = Q P, K_idx = K P for
               a seeded matrix P with orthonormal columns), 256 needles.
+* ``quest32k`` 32/8 heads, d=128, N=32768, B=128, bf16, top-16 per query head
+              scored by the K-min/K-max upper bound; the RBS recipe's clustered
+              keys with outliers, whose blocks the bound is designed to catch.
 
 The pages behind the method (RBS-Attention, "Uncertainty-gated selection for
 block-sparse attention", MiniMax Sparse Attention) evaluate on long-context
@@ -57,6 +60,7 @@ class Workload:
     group_shared: bool = False
     index_dim: int = 0
     seed: int = 0
+    backbone: str = "mean"          # "mean" (centroids) | "minmax" (K-min/K-max bound)
 
     @property
     def n_blocks(self) -> int:
@@ -100,6 +104,8 @@ CONFIGS = {
     "msa512k": Workload("msa512k", "msa", 64, 8, 524288, 128, 128, "bf16",
                         "topk", top_k=32, group_shared=True, index_dim=64,
                         seed=1005),
+    "quest32k": Workload("quest32k", "rbs", 32, 8, 32768, 128, 128, "bf16", "topk",
+                         top_k=16, seed=1006, backbone="minmax"),
 }
 
 # Reduced shapes of the same recipes, small enough for the CPU oracle to
@@ -117,6 +123,11 @@ SMALL = {
     "msa_small": CONFIGS["msa512k"].scaled(name="msa_small", n_q_heads=8,
                                            n_kv_heads=2, seq_len=8192 + 100,
                                            top_k=8),
+    "quest_small": CONFIGS["quest32k"].scaled(name="quest_small", n_q_heads=4,
+                                              n_kv_heads=2, seq_len=8192 + 50, top_k=8),
+    "quest_gate_small": CONFIGS["quest32k"].scaled(name="quest_gate_small", n_q_heads=4,
+                                                   n_kv_heads=2, seq_len=8192 + 50, top_k=8,
+                                                   gate_margin=0.05),
 }
 
 TORCH_DTYPE = {"bf16": torch.bfloat16, "fp32": torch.float32}

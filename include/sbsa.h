@@ -63,6 +63,13 @@ extern "C" {
 #define SBSA_CUMMASS 1 /* [RBS] base branch: shortest score-ranked prefix whose
                           softmax mass over the candidates reaches mass_threshold */
 
+/* ---- block-scoring backbones ([UGS] Metodologia step 1, Componibilidad) ---- */
+#define SBSA_BACKBONE_MEAN 0   /* centroid: s_j = q . c_j (SSA-style K-mean)          */
+#define SBSA_BACKBONE_MINMAX 1 /* per-coordinate upper bound from the block's K-min /
+                                  K-max: s_j = sum_d max(q_d min_jd, q_d max_jd),
+                                  the largest q.k over the block's coordinate box
+                                  (Quest-style K-max)                               */
+
 typedef struct sbsa_params {
   int n_q_heads;        /* Hq >= 1                                             */
   int n_kv_heads;       /* Hkv >= 1, divides Hq (GQA group G = Hq/Hkv)         */
@@ -84,6 +91,8 @@ typedef struct sbsa_params {
                            CUMMASS or rescue NB                                */
   float sm_scale;       /* attention logit scale; 0 => 1/sqrt(head_dim)       */
   float score_scale;    /* block-score scale;     0 => 1/sqrt(score dim)      */
+  int backbone;         /* SBSA_BACKBONE_MEAN | SBSA_BACKBONE_MINMAX; MINMAX
+                           excludes the rescue branch (which needs radii)    */
 } sbsa_params;
 
 /*
@@ -103,6 +112,19 @@ int sbsa_pool_blocks(const sbsa_params* p, const void* x, int n_heads, int dim, 
                      float* centroids, float* radii, void* stream);
 
 /*
+ * sbsa_pool_minmax -- [UGS] step 1 with the K-min / K-max backbone.
+ *   x       device [n_heads, N, dim], element type p->dtype.
+ *   minmax  device fp32 [n_heads, NB, 2, dim]: for block j, the coordinate-wise
+ *           minimum over the block's rows (t/B == j, t < N), then the maximum.
+ * Uses N and B from p; dim in {64, 128}.  Reads x once; exact (no rounding).
+ * Errors: SBSA_ERR_INVALID_ARG for null or misaligned pointers or n_heads < 1,
+ * SBSA_ERR_UNSUPPORTED for other dim or B; SBSA_ERR_CUDA on a launch failure.
+ * The pages have the backbone only by name; the table layout is this library's.
+ */
+int sbsa_pool_minmax(const sbsa_params* p, const void* x, int n_heads, int dim, float* minmax,
+                     void* stream);
+
+/*
  * sbsa_select -- [UGS] steps 1-5 on pooled tables; [RBS] base and rescue
  * branches with their union; [MSA] group-shared lists.
  *   q_cent   device fp32 [Hs, NB, ds]  pooled queries, Hs = group_shared ? Hkv : Hq
@@ -120,6 +142,9 @@ int sbsa_pool_blocks(const sbsa_params* p, const void* x, int n_heads, int dim, 
  */
 int sbsa_select(const sbsa_params* p, const float* q_cent, const float* k_cent,
                 const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags, void* stream);
+/* With p->backbone == SBSA_BACKBONE_MINMAX, k_cent is the [Hkv, NB, 2, ds]
+ * table of sbsa_pool_minmax and s_j = sum_d max(q_d min_jd, q_d max_jd) *
+ * score_scale; everything else is unchanged. */
 
 /*
  * sbsa_attend -- [RBS] sparse prefill attention; [MSA] main branch.

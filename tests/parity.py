@@ -102,9 +102,11 @@ def row_matches(gpu_ids, s, ub, i, w):
     return False
 
 
-def compare_lists(gpu_idx, gpu_cnt, oracle_idx, oracle_cnt, rows, qbar, c, r, w, kv_of_sel):
+def compare_lists(gpu_idx, gpu_cnt, oracle_idx, oracle_cnt, rows, qbar, c, r, w, kv_of_sel,
+                  minmax=None):
     """Returns (exact, tie) counts over ``rows``; raises AssertionError on a
-    difference the tie band does not explain."""
+    difference the tie band does not explain.  ``minmax`` = (kmin, kmax)
+    selects the upper-bound backbone's scores instead of the centroids'."""
     exact = tie = 0
     scale = 1.0 / math.sqrt(w.score_dim)
     for (hs, i) in rows:
@@ -114,7 +116,10 @@ def compare_lists(gpu_idx, gpu_cnt, oracle_idx, oracle_cnt, rows, qbar, c, r, w,
             exact += 1
             continue
         g = kv_of_sel(hs)
-        s = O.block_scores(qbar[hs, i], c[g], i, scale)
+        if minmax is None:
+            s = O.block_scores(qbar[hs, i], c[g], i, scale)
+        else:
+            s = O.block_bounds_minmax(qbar[hs, i], minmax[0][g], minmax[1][g], i, scale)
         ub = O.rescue_bounds(qbar[hs, i], c[g], r[g], i, scale) if w.rescue_tau is not None else None
         if not row_matches(gi, s, ub, i, w):
             raise AssertionError(f"row (head {hs}, block {i}): gpu {gi} vs oracle {oi}")

@@ -55,7 +55,7 @@ int main(void) {
   printf("size %zu\n", sizeof(sbsa_params));
   F(n_q_heads) F(n_kv_heads) F(seq_len) F(head_dim) F(block_size) F(dtype) F(select_mode)
   F(group_shared) F(index_dim) F(top_k) F(mass_threshold) F(rescue) F(rescue_tau) F(gate)
-  F(gate_margin) F(max_blocks) F(sm_scale) F(score_scale)
+  F(gate_margin) F(max_blocks) F(sm_scale) F(score_scale) F(backbone)
   return 0;
 }
 '''
@@ -110,6 +110,8 @@ def _attend(sb, p):
     (dict(top_k=4, gate_margin=0.05, max_blocks=5), 1),   # gated needs 2k+1 = 9
     (dict(select_mode="cummass", mass_threshold=0.9, max_blocks=5), 1),  # needs NB
     (dict(sm_scale=-1.0), 1),
+    (dict(backbone=2), 1),                       # no such backbone
+    (dict(select_mode="cummass", mass_threshold=0.9, rescue_tau=5.0, backbone="minmax"), 1),
 ])
 def test_invalid_parameters_are_rejected_before_launch(sb, mutate, code):
     p = _valid(sb, **mutate)
@@ -140,6 +142,26 @@ def test_pool_argument_checks(sb):
     assert sb.lib.sbsa_pool_blocks(ctypes.byref(p), FAKE, 3, 128, 2, FAKE, None, None) == 1
     assert sb.lib.sbsa_pool_blocks(ctypes.byref(p), FAKE, 4, 96, 1, FAKE, None, None) == 2
     assert sb.lib.sbsa_pool_blocks(ctypes.byref(p), FAKE, 4, 128, 2, FAKE, FAKE, None) == 1
+
+
+def test_pool_minmax_argument_checks(sb):
+    p = _valid(sb)
+    assert sb.lib.sbsa_pool_minmax(ctypes.byref(p), None, 2, 128, FAKE, None) == 1
+    assert sb.lib.sbsa_pool_minmax(ctypes.byref(p), FAKE, 0, 128, FAKE, None) == 1
+    assert sb.lib.sbsa_pool_minmax(ctypes.byref(p), FAKE, 2, 96, FAKE, None) == 2
+    assert sb.lib.sbsa_pool_minmax(ctypes.byref(p), FAKE, 2, 128,
+                                   ctypes.c_void_p((1 << 20) + 4), None) == 1
+
+
+def test_minmax_backbone_doubles_the_key_table_in_the_workspace(sb):
+    mean = _valid(sb)
+    mm = _valid(sb, backbone="minmax")
+    nb = mean.n_blocks
+
+    def r256(x):
+        return (x + 255) // 256 * 256
+    extra = r256(2 * 2 * nb * 128 * 4) - r256(2 * nb * 128 * 4)
+    assert sb.workspace_bytes(mm) == sb.workspace_bytes(mean) + extra
 
 
 def test_fp32_attention_is_limited_to_d64_b64(sb):

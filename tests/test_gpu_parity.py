@@ -14,7 +14,8 @@ from block_sparse_attention_sbsa_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-SMALL_NAMES = ["tiny", "gqa_small", "rbs_small", "gate_small", "msa_small"]
+SMALL_NAMES = ["tiny", "gqa_small", "rbs_small", "gate_small", "msa_small", "quest_small",
+               "quest_gate_small"]
 
 
 @pytest.fixture(scope="module")
@@ -29,7 +30,7 @@ def _oracle_prefill(w, data, **kw):
     return O.prefill(data["q"], data["k"], data["v"], block=w.block_size, mode=w.select_mode,
                      top_k_=w.top_k, mass=w.mass_threshold, margin=w.gate_margin,
                      tau=w.rescue_tau, group_shared=w.group_shared, q_idx=data["q_idx"],
-                     k_idx=data["k_idx"], max_blocks=w.max_blocks, **kw)
+                     k_idx=data["k_idx"], max_blocks=w.max_blocks, backbone=w.backbone, **kw)
 
 
 @functools.lru_cache(maxsize=None)
@@ -60,6 +61,11 @@ def test_pool_matches_oracle(sb, name):
     qs = d["q_idx"] if w.index_dim else d["q"]
     c, r = sb.pool_blocks(p, ks, group=1, radius=True)
     qb, _ = sb.pool_blocks(p, qs, group=w.group if w.group_shared else 1)
+    if w.backbone == "minmax":
+        # coordinate-wise min and max of bf16/fp32 values: exact
+        mm = sb.pool_minmax(p, ks).cpu().numpy()
+        np.testing.assert_array_equal(mm[:, :, 0], ref["minmax"][0])
+        np.testing.assert_array_equal(mm[:, :, 1], ref["minmax"][1])
     torch.cuda.synchronize()
     np.testing.assert_allclose(c.cpu().numpy(), ref["c"], rtol=1e-5, atol=2e-5)
     np.testing.assert_allclose(qb.cpu().numpy(), ref["qbar"], rtol=1e-5, atol=2e-5)
@@ -74,12 +80,15 @@ def test_select_on_oracle_tables(sb, name):
     w, data, ref = small_case(name)
     p = sb.params_for(w)
     qc = torch.tensor(ref["qbar"], dtype=torch.float32, device="cuda")
-    kc = torch.tensor(ref["c"], dtype=torch.float32, device="cuda")
+    if w.backbone == "minmax":
+        kc = torch.tensor(np.stack(ref["minmax"], axis=2), dtype=torch.float32, device="cuda")
+    else:
+        kc = torch.tensor(ref["c"], dtype=torch.float32, device="cuda")
     kr = torch.tensor(ref["r"], dtype=torch.float32, device="cuda")
     idx, cnt, flags = sb.select(p, qc, kc, kr if w.rescue_tau is not None else None)
     idx, cnt, flags = idx.cpu().numpy(), cnt.cpu().numpy(), flags.cpu().numpy()
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
-                                  ref["c"], ref["r"], w, _kv_of_sel(w))
+                                  ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"])
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # padding and flags
     for hs in range(w.n_sel_heads):
@@ -115,7 +124,7 @@ def test_prefill_end_to_end(sb, name):
     assert sb.get_status() == sb.OK
     idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
-                                  ref["c"], ref["r"], w, _kv_of_sel(w))
+                                  ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"])
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # outputs on query rows whose lists match the oracle exactly
     o = o.float().cpu().numpy()
@@ -141,7 +150,7 @@ def test_gate_fires_on_the_planted_rows(sb):
 
 # ------------------------------------------------------------- full sizes
 
-FULL = ["gqa32k", "rbs128k", "gate64k", "msa512k"]
+FULL = ["gqa32k", "rbs128k", "gate64k", "msa512k", "quest32k"]
 
 
 def _sample_blocks(w, meta, count):
@@ -172,6 +181,7 @@ def test_full_size_sampled(sb, name):
     c, r = O.pool_keys(ks, w.block_size, with_radius=w.rescue_tau is not None)
     if r is None:
         r = np.zeros(c.shape[:2])
+    mmx = O.pool_keys_minmax(ks, w.block_size) if w.backbone == "minmax" else None
     nb = w.n_blocks
     qrows = torch.cat([qs[:, i * w.block_size:(i + 1) * w.block_size] for i in blocks], dim=1).cpu()
     # pooled queries of the sampled blocks only
@@ -185,7 +195,7 @@ def test_full_size_sampled(sb, name):
     idx, cnt, flags = O.select(qbar, c, r, block_count=nb, mode=w.select_mode, top_k_=w.top_k,
                                mass=w.mass_threshold, margin=w.gate_margin, tau=w.rescue_tau,
                                scale=1.0 / math.sqrt(w.score_dim), kv_of_sel=_kv_of_sel(w),
-                               max_blocks=w.max_blocks, rows=sel_rows)
+                               max_blocks=w.max_blocks, rows=sel_rows, minmax=mmx)
     gidx = call.idx[:, blocks].cpu().numpy()
     gcnt = call.cnt[:, blocks].cpu().numpy()
     gi_full = np.full((w.n_sel_heads, nb, w.max_blocks), -1, dtype=np.int32)
@@ -193,7 +203,7 @@ def test_full_size_sampled(sb, name):
     gi_full[:, blocks] = gidx
     gc_full[:, blocks] = gcnt
     exact, tie = PT.compare_lists(gi_full, gc_full, idx, cnt, sel_rows, qbar, c, r, w,
-                                  _kv_of_sel(w))
+                                  _kv_of_sel(w), minmax=mmx)
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # outputs of the sampled blocks whose lists match (all query heads; two
     # per group for the 64-head workload); keys/values converted once per

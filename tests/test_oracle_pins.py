@@ -308,7 +308,8 @@ def _check_lists(idx, cnt, nb):
             assert np.all(idx[h, i, c:] == -1)
 
 
-@pytest.mark.parametrize("name", ["tiny", "gqa_small", "rbs_small", "gate_small", "msa_small"])
+@pytest.mark.parametrize("name", ["tiny", "gqa_small", "rbs_small", "gate_small", "msa_small",
+                                  "quest_small", "quest_gate_small"])
 def test_small_workload_lists_are_causal_sorted_padded(name):
     w = W.SMALL[name]
     data = W.generate(w)
@@ -316,7 +317,7 @@ def test_small_workload_lists_are_causal_sorted_padded(name):
                     top_k_=w.top_k, mass=w.mass_threshold, margin=w.gate_margin,
                     tau=w.rescue_tau, group_shared=w.group_shared, q_idx=data["q_idx"],
                     k_idx=data["k_idx"], max_blocks=w.max_blocks,
-                    attend_rows=[(0, w.n_blocks - 1)])
+                    attend_rows=[(0, w.n_blocks - 1)], backbone=w.backbone)
     _check_lists(res["idx"], res["cnt"], w.n_blocks)
 
 
