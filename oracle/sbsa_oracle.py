@@ -43,6 +43,13 @@ candidates and keeps the shortest prefix of the ranked order whose mass
 reaches the threshold; the rescue test is (q.c + |q| r) * scale > tau.
 The K-min/K-max backbone bounds q.k over the block's keys coordinate by
 coordinate: sum_d max(q_d * min_d, q_d * max_d), scaled like the mean score.
+The page's own gate (Metodologia steps 3-5): the normalised cut margin
+sigma = (s_(k-1) - s_(k)) / (s_(0) - s_(k)) on the descending 0-based order
+(0 when s_(0) = s_(k)), defined for rows with more than k candidates; its
+mean over the selection heads gives one value per query tile; the floor(q T)
+eligible tiles with the smallest mean (lower tile first on equal means; T
+eligible tiles) fire -- the empirical percentile q of the layer -- and take
+the top rho*k blocks in every head, the others the top k.
 """
 from __future__ import annotations
 
@@ -194,6 +201,27 @@ def gate(s, k: int, margin: float):
     return bool(gap < thr), float(gap), float(thr)
 
 
+def cut_margin(s, k: int) -> float:
+    """Normalised cut margin of a row with more than k candidates:
+    (s_(k-1) - s_(k)) / (s_(0) - s_(k)) with s_(m) the m-th largest (0-based),
+    in float64 from the row's (float32) scores; 0 when s_(0) = s_(k)."""
+    s64 = np.asarray(s, dtype=np.float64)
+    if len(s64) <= k:
+        raise ValueError("cut margin needs more than k candidates")
+    order = ranked(s64)
+    top, last, first_out = s64[order[0]], s64[order[k - 1]], s64[order[k]]
+    if top == first_out:
+        return 0.0
+    return float((last - first_out) / (top - first_out))
+
+
+def percentile_fire(sbar: dict, q: float) -> set:
+    """Tiles that fire: the floor(q T) tiles with the smallest head-averaged
+    margin among the T eligible ones (lower tile index first on ties)."""
+    order = sorted(sbar, key=lambda i: (sbar[i], i))
+    return set(order[:int(math.floor(q * len(order)))])
+
+
 def cumulative_mass(s, mass: float):
     """Base branch with its own threshold: p = softmax over the candidates;
     keep the shortest prefix of the ranked order whose mass reaches ``mass``.
@@ -211,13 +239,18 @@ def cumulative_mass(s, mass: float):
 
 
 def select_row(s, i: int, *, mode: str, top_k_: int = 0, mass: float = 0.0,
-               margin=None, ub=None, tau=None):
+               margin=None, ub=None, tau=None, budget=None):
     """Block list of query block i: base branch (top-k, gated top-k or
     cumulative mass), united with the rescue branch, plus the diagonal block
-    i, ascending.  Returns (ids, flags)."""
+    i, ascending.  ``budget`` overrides k (the percentile gate's rho*k for a
+    fired tile).  Returns (ids, flags)."""
     flags = 0
     n = i
-    if mode == "topk":
+    if mode == "topk" and budget is not None:
+        base = set(top_k(s, budget).tolist())
+        if budget > top_k_:
+            flags |= FLAG_GATE
+    elif mode == "topk":
         kk = top_k_
         if margin is not None and n > top_k_:
             fired, _, _ = gate(s, top_k_, margin)
@@ -241,7 +274,7 @@ def select_row(s, i: int, *, mode: str, top_k_: int = 0, mass: float = 0.0,
 
 def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
            mass: float = 0.0, margin=None, tau=None, scale: float,
-           kv_of_sel=None, max_blocks: int, rows=None, minmax=None):
+           kv_of_sel=None, max_blocks: int, rows=None, minmax=None, sigma_gate=None):
     """Lists for every selection head hs and query block i (or the (hs, i)
     pairs in ``rows``).  ``qbar`` is [Hs, NB, d_s] and ``c``/``r`` are the key
     tables [Hkv, NB, ...]; ``kv_of_sel(hs)`` gives the kv head whose key table
@@ -253,15 +286,32 @@ def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
     cnt = np.zeros((hs_n, nb), dtype=np.int32)
     flags = np.zeros((hs_n, nb), dtype=np.uint8)
     pairs = rows if rows is not None else [(h, i) for h in range(hs_n) for i in range(nb)]
-    for (h, i) in pairs:
+
+    def scores(h, i):
         g = kv_of_sel(h)
         if minmax is None:
-            s = block_scores(qbar[h, i], c[g], i, scale)
-        else:
-            s = block_bounds_minmax(qbar[h, i], minmax[0][g], minmax[1][g], i, scale)
+            return block_scores(qbar[h, i], c[g], i, scale)
+        return block_bounds_minmax(qbar[h, i], minmax[0][g], minmax[1][g], i, scale)
+
+    fired = set()
+    if sigma_gate is not None:
+        if mode != "topk" or margin is not None:
+            raise ValueError("the percentile gate applies to plain top-k")
+        q, rho = sigma_gate
+        sbar = {}
+        for i in range(top_k_ + 1, nb):          # tiles with more than k candidates
+            tot = 0.0
+            for h in range(hs_n):                 # head order, one sum
+                tot += cut_margin(scores(h, i), top_k_)
+            sbar[i] = tot / hs_n
+        fired = percentile_fire(sbar, q)
+    for (h, i) in pairs:
+        g = kv_of_sel(h)
+        s = scores(h, i)
         ub = rescue_bounds(qbar[h, i], c[g], r[g], i, scale) if tau is not None else None
+        budget = sigma_gate[1] * top_k_ if i in fired else None
         ids, fl = select_row(s, i, mode=mode, top_k_=top_k_, mass=mass,
-                             margin=margin, ub=ub, tau=tau)
+                             margin=margin, ub=ub, tau=tau, budget=budget)
         if len(ids) > max_blocks:
             raise ValueError("selection wider than max_blocks")
         idx[h, i, :len(ids)] = ids
@@ -359,7 +409,8 @@ def attend_dense_masked(q, k, v, idx, cnt, *, block: int, scale: float,
 def prefill(q, k, v, *, block: int, mode: str, top_k_: int = 0,
             mass: float = 0.0, margin=None, tau=None, group_shared: bool = False,
             q_idx=None, k_idx=None, max_blocks: int, scale=None,
-            score_scale=None, sel_rows=None, attend_rows=None, backbone: str = "mean"):
+            score_scale=None, sel_rows=None, attend_rows=None, backbone: str = "mean",
+            sigma_gate=None):
     """Selection tables and lists from the index tensors (q_idx/k_idx when
     given, else q/k), then attention over the lists.  ``sel_rows`` restricts
     selection to (hs, i) pairs, ``attend_rows`` restricts attention to
@@ -393,7 +444,7 @@ def prefill(q, k, v, *, block: int, mode: str, top_k_: int = 0,
     idx, cnt, flags = select(qbar, c, r, block_count=nb, mode=mode, top_k_=top_k_,
                              mass=mass, margin=margin, tau=tau, scale=score_scale,
                              kv_of_sel=kv_of_sel, max_blocks=max_blocks,
-                             rows=sel_rows, minmax=minmax)
+                             rows=sel_rows, minmax=minmax, sigma_gate=sigma_gate)
     out = attend(q, k, v, idx, cnt, block=block, scale=scale,
                  group_shared=group_shared, rows=attend_rows)
     return dict(c=c, r=r, qbar=qbar, idx=idx, cnt=cnt, flags=flags, o=out,

@@ -446,3 +446,89 @@ def test_minmax_backbone_rejects_the_rescue_branch():
     with pytest.raises(ValueError):
         O.prefill(x, x, x, block=32, mode="cummass", mass=0.9, tau=1.0, max_blocks=2,
                   backbone="minmax")
+
+
+# --------------------------------------------------------------------------
+# The page's own gate (uncertainty-gated page, Metodologia steps 3-5):
+# sigma = (s_(k-1) - s_(k)) / (s_(0) - s_(k)), head average per tile,
+# empirical percentile q, expansion to top rho*k
+# --------------------------------------------------------------------------
+
+def test_cut_margin_closed_forms():
+    # three patches 10, 9.9, 9.8 and k = 2: (9.9 - 9.8) / (10 - 9.8) = 1/2
+    assert O.cut_margin(np.array([9.8, 10.0, 9.9]), 2) == pytest.approx(0.5, rel=1e-6)
+    # an exact tie at the cut: ambiguous
+    assert O.cut_margin(np.array([5.0, 3.0, 3.0, 1.0]), 2) == 0.0
+    # all kept scores equal and the first dropped below: decisive
+    assert O.cut_margin(np.array([4.0, 4.0, 4.0, 1.0]), 3) == 1.0
+    # everything tied: 0 (no cut at all)
+    assert O.cut_margin(np.array([2.0, 2.0, 2.0]), 1) == 0.0
+    # k = 1 normalises the gap by itself
+    assert O.cut_margin(np.array([9.9, 9.8]), 1) == 1.0
+    with pytest.raises(ValueError):
+        O.cut_margin(np.array([1.0, 2.0]), 2)
+
+
+def test_cut_margin_lies_in_unit_interval_and_ignores_affine_rescaling():
+    rng = np.random.default_rng(31)
+    for _ in range(200):
+        s = rng.standard_normal(rng.integers(3, 40)).astype(np.float32)
+        k = int(rng.integers(1, len(s)))
+        m = O.cut_margin(s, k)
+        assert 0.0 <= m <= 1.0
+        assert O.cut_margin(3.0 * s.astype(np.float64) + 7.0, k) == pytest.approx(m, abs=1e-6)
+
+
+def _sigma_case(seed=32):
+    rng = np.random.default_rng(seed)
+    hs, nb, d = 3, 20, 8
+    qbar = rng.standard_normal((hs, nb, d))
+    c = rng.standard_normal((hs, nb, d))
+    r = np.zeros((hs, nb))
+    return qbar, c, r
+
+
+def _sel(qbar, c, r, **kw):
+    base = dict(block_count=qbar.shape[1], mode="topk", scale=0.5, kv_of_sel=lambda h: h,
+                max_blocks=qbar.shape[1])
+    base.update(kw)
+    return O.select(qbar, c, r, **base)
+
+
+def test_percentile_gate_extremes_reduce_to_plain_top_k():
+    qbar, c, r = _sigma_case()
+    k = 3
+    none = _sel(qbar, c, r, top_k_=k, sigma_gate=(0.0, 2))
+    plain = _sel(qbar, c, r, top_k_=k)
+    assert np.array_equal(none[0], plain[0]) and not (none[2] & O.FLAG_GATE).any()
+    every = _sel(qbar, c, r, top_k_=k, sigma_gate=(1.0, 2))
+    double = _sel(qbar, c, r, top_k_=2 * k)
+    assert np.array_equal(every[0], double[0])
+    fired_rows = (every[2] & O.FLAG_GATE) != 0
+    assert fired_rows[:, k + 1:].all() and not fired_rows[:, :k + 1].any()
+
+
+@pytest.mark.parametrize("q", [0.25, 0.5, 0.8])
+def test_percentile_gate_fires_the_floor_q_t_most_ambiguous_tiles(q):
+    qbar, c, r = _sigma_case(33)
+    k, rho = 2, 3
+    hs, nb = qbar.shape[:2]
+    idx, cnt, flags = _sel(qbar, c, r, top_k_=k, sigma_gate=(q, rho))
+    eligible = list(range(k + 1, nb))
+    # the head-averaged margin of every eligible tile, recomputed from its definition
+    sbar = {i: np.mean([O.cut_margin(O.block_scores(qbar[h, i], c[h], i, 0.5), k)
+                        for h in range(hs)]) for i in eligible}
+    fired = [i for i in eligible if flags[0, i] & O.FLAG_GATE]
+    assert len(fired) == int(math.floor(q * len(eligible)))
+    # every head of a fired tile fires, and takes rho*k blocks plus the diagonal
+    for i in eligible:
+        assert len({bool(flags[h, i] & O.FLAG_GATE) for h in range(hs)}) == 1
+        want = min(rho * k, i) + 1 if i in fired else k + 1
+        assert all(cnt[h, i] == want for h in range(hs))
+    rest = [i for i in eligible if i not in fired]
+    if fired and rest:
+        assert max(sbar[i] for i in fired) <= min(sbar[i] for i in rest) + 1e-12
+
+
+def test_percentile_gate_breaks_equal_margins_by_lower_tile():
+    assert O.percentile_fire({5: 0.2, 3: 0.2, 9: 0.1, 7: 0.9}, 0.5) == {9, 3}
