@@ -36,6 +36,13 @@ struct SelectArgs {
   int kmax;
   int mode;          // SBSA_TOPK | SBSA_CUMMASS
   int minmax;        // 1: upper-bound scores from the min/max table
+  // percentile gate (SBSA_GATE_PERCENTILE): pass 1 writes top-k lists and the
+  // per-row cut margins, pass 2 rewrites the rows of fired tiles with top
+  // rho*k; pass 0 is the ordinary single pass
+  int pass;
+  int rho;
+  double* sigma;        // [Hs, NB] cut margins (NaN: no cut), written by pass 1
+  const uint8_t* fire;  // [NB] 1 for fired tiles, read by pass 2
   int top_k;
   float mass;
   int gate;
@@ -45,6 +52,11 @@ struct SelectArgs {
   float score_scale;
   int* status;
 };
+
+// The percentile gate's tile decisions: mean margin per tile over the Hs
+// heads, the floor(q T) smallest of the T tiles with more than k candidates.
+cudaError_t launch_gate_tiles(const double* sigma, uint8_t* fire, int n_sel_heads, int nb,
+                              int top_k, float quantile, cudaStream_t stream);
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 

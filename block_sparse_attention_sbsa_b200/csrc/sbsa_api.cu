@@ -58,8 +58,13 @@ int validate(const sbsa_params* p, Derived* d) {
   if (p->select_mode == SBSA_CUMMASS &&
       !(p->mass_threshold > 0.f && p->mass_threshold <= 1.f))
     return SBSA_ERR_INVALID_ARG;
+  if (p->gate != 0 && p->gate != SBSA_GATE_GAP && p->gate != SBSA_GATE_PERCENTILE)
+    return SBSA_ERR_INVALID_ARG;
   if (p->gate && p->select_mode != SBSA_TOPK) return SBSA_ERR_INVALID_ARG;
-  if (p->gate && !(p->gate_margin >= 0.f && std::isfinite(p->gate_margin)))
+  if (p->gate == SBSA_GATE_GAP && !(p->gate_margin >= 0.f && std::isfinite(p->gate_margin)))
+    return SBSA_ERR_INVALID_ARG;
+  if (p->gate == SBSA_GATE_PERCENTILE &&
+      (!(p->gate_quantile >= 0.f && p->gate_quantile <= 1.f) || p->gate_rho < 1))
     return SBSA_ERR_INVALID_ARG;
   if (p->rescue && std::isnan(p->rescue_tau)) return SBSA_ERR_INVALID_ARG;
   if (p->backbone != SBSA_BACKBONE_MEAN && p->backbone != SBSA_BACKBONE_MINMAX)
@@ -75,12 +80,17 @@ int validate(const sbsa_params* p, Derived* d) {
   if (p->select_mode == SBSA_CUMMASS || p->rescue) {
     o.need_kmax = o.nb;
   } else {
-    long long budget = p->gate ? 2LL * p->top_k : (long long)p->top_k;
+    long long budget = p->top_k;
+    if (p->gate == SBSA_GATE_GAP) budget = 2LL * p->top_k;
+    if (p->gate == SBSA_GATE_PERCENTILE) budget = (long long)p->gate_rho * p->top_k;
     if (budget > o.nb - 1) budget = o.nb - 1;
     o.need_kmax = (int)budget + 1;
   }
   if (p->max_blocks < o.need_kmax) return SBSA_ERR_INVALID_ARG;
   if ((long long)p->n_q_heads * o.nb > 0x7FFFFFFFLL) return SBSA_ERR_UNSUPPORTED;
+  // the percentile gate's tile means are held in one CTA's shared memory
+  if (p->gate == SBSA_GATE_PERCENTILE && (size_t)o.nb * sizeof(double) > 227 * 1024)
+    return SBSA_ERR_UNSUPPORTED;
   o.sm_scale = p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt((float)p->head_dim);
   o.score_scale = p->score_scale > 0.f ? p->score_scale : 1.0f / std::sqrt((float)o.ds);
   if (d) *d = o;
@@ -94,8 +104,19 @@ int attend_supported(const sbsa_params* p) {
 }
 
 struct WsLayout {
-  size_t qc, kc, kr, idx, cnt, flags, total;
+  size_t qc, kc, kr, idx, cnt, flags, sigma, fire, total;
 };
+
+// Scratch of the percentile gate: per-row margins (double) and per-tile
+// decisions, placed from offset `off`.
+size_t gate_scratch(const sbsa_params* p, const Derived& d, size_t off, size_t* sigma,
+                    size_t* fire) {
+  *sigma = off;
+  if (p->gate == SBSA_GATE_PERCENTILE) off = round_up(off + (size_t)d.hs * d.nb * 8, 256);
+  *fire = off;
+  if (p->gate == SBSA_GATE_PERCENTILE) off = round_up(off + (size_t)d.nb, 256);
+  return off;
+}
 
 WsLayout layout(const sbsa_params* p, const Derived& d, bool lists) {
   WsLayout w{};
@@ -113,6 +134,7 @@ WsLayout layout(const sbsa_params* p, const Derived& d, bool lists) {
   off = round_up(off + (lists ? (size_t)d.hs * d.nb * 4 : 0), 256);
   w.flags = off;
   off = round_up(off + (lists ? (size_t)d.hs * d.nb : 0), 256);
+  off = gate_scratch(p, d, off, &w.sigma, &w.fire);
   w.total = off;
   return w;
 }
@@ -137,13 +159,32 @@ SelectArgs select_args(const sbsa_params* p, const Derived& d, const float* qc, 
   a.minmax = p->backbone == SBSA_BACKBONE_MINMAX ? 1 : 0;
   a.top_k = p->top_k;
   a.mass = p->mass_threshold;
-  a.gate = p->gate ? 1 : 0;
+  a.gate = p->gate == SBSA_GATE_GAP ? 1 : 0;
+  a.rho = p->gate_rho;
   a.margin = p->gate_margin;
   a.rescue = p->rescue ? 1 : 0;
   a.tau = p->rescue_tau;
   a.score_scale = d.score_scale;
   a.status = device_status_ptr();
   return a;
+}
+
+// The selection on a stream: one launch, or for the percentile gate the
+// three of it (top-k lists and margins, tile decisions, fired tiles again).
+int run_select(const sbsa_params* p, const Derived& d, SelectArgs a, unsigned char* scratch,
+               size_t sigma_off, size_t fire_off, cudaStream_t s) {
+  if (p->gate != SBSA_GATE_PERCENTILE) return cuda_code(launch_select(a, s));
+  double* sigma = reinterpret_cast<double*>(scratch + sigma_off);
+  uint8_t* fire = scratch + fire_off;
+  a.sigma = sigma;
+  a.fire = fire;
+  a.pass = 1;
+  int rc = cuda_code(launch_select(a, s));
+  if (rc) return rc;
+  rc = cuda_code(launch_gate_tiles(sigma, fire, d.hs, d.nb, p->top_k, p->gate_quantile, s));
+  if (rc) return rc;
+  a.pass = 2;
+  return cuda_code(launch_select(a, s));
 }
 
 AttendArgs attend_args(const sbsa_params* p, const Derived& d, const void* q, const void* k,
@@ -175,7 +216,7 @@ using namespace sbsa;
 
 extern "C" {
 
-int sbsa_version(void) { return 101; }
+int sbsa_version(void) { return 102; }
 
 const char* sbsa_status_string(int code) {
   switch (code) {
@@ -228,9 +269,37 @@ int sbsa_select(const sbsa_params* p, const float* q_cent, const float* k_cent,
   if (!q_cent || !k_cent || !idx || !cnt) return SBSA_ERR_INVALID_ARG;
   if (p->rescue && !k_radius) return SBSA_ERR_INVALID_ARG;
   if (!aligned16(q_cent) || !aligned16(k_cent)) return SBSA_ERR_INVALID_ARG;
+  if (p->gate == SBSA_GATE_PERCENTILE) return SBSA_ERR_WORKSPACE;  // use sbsa_select_ws
   SelectArgs a = select_args(p, d, q_cent, k_cent, p->rescue ? k_radius : nullptr, idx, cnt,
                              flags);
   return cuda_code(launch_select(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t sbsa_select_workspace_bytes(const sbsa_params* p) {
+  Derived d;
+  if (validate(p, &d) != SBSA_OK) return 0;
+  size_t sigma, fire;
+  return gate_scratch(p, d, 0, &sigma, &fire);
+}
+
+int sbsa_select_ws(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                   const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  Derived d;
+  int rc = validate(p, &d);
+  if (rc) return rc;
+  if (!q_cent || !k_cent || !idx || !cnt) return SBSA_ERR_INVALID_ARG;
+  if (p->rescue && !k_radius) return SBSA_ERR_INVALID_ARG;
+  if (!aligned16(q_cent) || !aligned16(k_cent)) return SBSA_ERR_INVALID_ARG;
+  size_t sigma, fire;
+  const size_t need = gate_scratch(p, d, 0, &sigma, &fire);
+  if (need && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+               ws_bytes < need))
+    return SBSA_ERR_WORKSPACE;
+  SelectArgs a = select_args(p, d, q_cent, k_cent, p->rescue ? k_radius : nullptr, idx, cnt,
+                             flags);
+  return run_select(p, d, a, static_cast<unsigned char*>(workspace), sigma, fire,
+                    static_cast<cudaStream_t>(stream));
 }
 
 int sbsa_attend(const sbsa_params* p, const void* q, const void* k, const void* v,
@@ -288,7 +357,7 @@ int sbsa_prefill(const sbsa_params* p, const void* q, const void* k, const void*
   };
   rc = cuda_code(launch_pool(p->dtype, d.ds, p->seq_len, p->block_size, jobs, 2, s));
   if (rc) return rc;
-  rc = cuda_code(launch_select(select_args(p, d, qc, kc, kr, idx, cnt, flags), s));
+  rc = run_select(p, d, select_args(p, d, qc, kc, kr, idx, cnt, flags), ws, w.sigma, w.fire, s);
   if (rc) return rc;
   return launch_attend(attend_args(p, d, q, k, v, idx, cnt, o), s);
 }

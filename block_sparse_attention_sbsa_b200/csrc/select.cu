@@ -305,6 +305,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
   const int rows = min(R, a.nb - i0);
   const int g = hs / a.kv_div;
   const int jend = i0 + rows - 1;  // candidates needed: j < jend
+  if (a.pass == 2) {
+    // nothing to redo unless one of this CTA's query blocks fired
+    int any = 0;
+    for (int r = tid; r < rows; r += kSelThreads) any |= a.fire[i0 + r];
+    if (!__syncthreads_or(any)) return;
+  }
 
   for (int e = tid; e < R * DS; e += kSelThreads) {
     const int r = e / DS;
@@ -388,12 +394,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
     uint8_t flag = 0;
     if (a.mode == SBSA_TOPK) {
       int kk = a.top_k;
+      if (a.pass == 2) {
+        // percentile gate, second pass: only the rows of fired tiles change
+        if (!a.fire[i]) continue;
+        kk = a.rho * a.top_k;
+        flag |= 1;
+      }
       if (n <= kk) {
         select_all = true;
+        if (a.pass == 1 && lane == 0) a.sigma[(size_t)hs * a.nb + i] = __longlong_as_double(0x7FF8000000000000ll);
       } else {
-        // every rank the row may need (k, k+1 for the gap test, 2k when the
-        // gate fires) lies in the short list when it fits
-        const int need = min(n, (a.gate ? 2 * a.top_k : a.top_k) + 1);
+        // every rank the row may need (k, k+1 for the gap test or the cut
+        // margin, 2k when the gap gate fires) lies in the short list when it fits
+        const int need = min(n, (a.gate ? 2 * a.top_k : kk) + 1);
         int m = 0;
         bool short_ok = false;
         if (need <= 32) short_ok = topk_short<1>(s, n, need, hist32, sbuf, kShortCap, &m);
@@ -407,6 +420,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
         int n_gt, n_eq;
         vkey = rank_key(kk - 1, &n_gt, &n_eq);
         take_eq = kk - n_gt;
+        if (a.pass == 1) {
+          // cut margin (s_(k-1) - s_(k)) / (s_(0) - s_(k)), 0-based ranks,
+          // in double from the float scores; 0 when s_(0) = s_(k)
+          const float last = key_float(vkey);
+          float first_out = last;
+          if (n_gt + n_eq < kk + 1) {
+            int g1, e1;
+            first_out = key_float(rank_key(kk, &g1, &e1));
+          }
+          int g0, e0;
+          const float top = key_float(rank_key(0, &g0, &e0));
+          const double sg = top == first_out
+                                ? 0.0
+                                : ((double)last - (double)first_out) / ((double)top - (double)first_out);
+          if (lane == 0) a.sigma[(size_t)hs * a.nb + i] = sg;
+        }
         if (a.gate) {
           // s_(k) and s_(k+1); population std of the candidates (double)
           const float sk = key_float(vkey);
@@ -573,6 +602,37 @@ cudaError_t launch_rows(const SelectArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Percentile gate, tile decisions: the mean cut margin of each query tile
+// over the selection heads (summed in head order, double), then the
+// floor(q T) smallest of the T tiles with more than k candidates fire, lower
+// tile first on equal means.  One CTA; the means live in shared memory.
+__global__ void __launch_bounds__(1024) gate_tiles_kernel(const double* sigma, uint8_t* fire,
+                                                          int n_sel_heads, int nb, int top_k,
+                                                          float quantile) {
+  extern __shared__ double sbar[];
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    double tot = 0.0;
+    for (int h = 0; h < n_sel_heads; ++h) tot += sigma[(size_t)h * nb + i];
+    sbar[i] = tot / (double)n_sel_heads;
+  }
+  __syncthreads();
+  const int t_eligible = nb - 1 - top_k > 0 ? nb - 1 - top_k : 0;
+  const int n_fire = (int)floor((double)quantile * (double)t_eligible);
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    uint8_t f = 0;
+    if (i > top_k && n_fire > 0) {
+      const double si = sbar[i];
+      int rank = 0;
+      for (int j = top_k + 1; j < nb; ++j) {
+        const double sj = sbar[j];
+        rank += (sj < si || (sj == si && j < i)) ? 1 : 0;
+      }
+      f = rank < n_fire ? 1 : 0;
+    }
+    fire[i] = f;
+  }
+}
+
 template <int DS>
 cudaError_t launch_ds(const SelectArgs& a, cudaStream_t stream) {
   // rows per CTA: as many (up to 16) as the score rows allow in shared memory;
@@ -587,6 +647,18 @@ cudaError_t launch_ds(const SelectArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t launch_gate_tiles(const double* sigma, uint8_t* fire, int n_sel_heads, int nb,
+                              int top_k, float quantile, cudaStream_t stream) {
+  const size_t smem = (size_t)nb * sizeof(double);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(gate_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  gate_tiles_kernel<<<1, 1024, smem, stream>>>(sigma, fire, n_sel_heads, nb, top_k, quantile);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   return a.ds == 128 ? launch_ds<128>(a, stream) : launch_ds<64>(a, stream);

@@ -22,9 +22,11 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_
 BF16, FP32 = 0, 1
 TOPK, CUMMASS = 0, 1
 BACKBONE_MEAN, BACKBONE_MINMAX = 0, 1
+GATE_GAP, GATE_PERCENTILE = 1, 2
 FLAG_GATE, FLAG_RESCUE = 1, 2
 
-SYMBOLS = ["sbsa_pool_blocks", "sbsa_pool_minmax", "sbsa_select", "sbsa_attend", "sbsa_prefill",
+SYMBOLS = ["sbsa_pool_blocks", "sbsa_pool_minmax", "sbsa_select", "sbsa_select_ws",
+           "sbsa_select_workspace_bytes", "sbsa_attend", "sbsa_prefill",
            "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string",
            "sbsa_version", "sbsa_debug_wait_timeout"]
 
@@ -56,6 +58,8 @@ class Params(ctypes.Structure):
         ("sm_scale", ctypes.c_float),
         ("score_scale", ctypes.c_float),
         ("backbone", ctypes.c_int),
+        ("gate_quantile", ctypes.c_float),
+        ("gate_rho", ctypes.c_int),
     ]
 
     @property
@@ -83,6 +87,9 @@ def _load() -> ctypes.CDLL:
     lib.sbsa_pool_blocks.argtypes = [P, vp, ci, ci, ci, f32p, f32p, vp]
     lib.sbsa_pool_minmax.argtypes = [P, vp, ci, ci, f32p, vp]
     lib.sbsa_select.argtypes = [P, f32p, f32p, f32p, i32p, i32p, u8p, vp]
+    lib.sbsa_select_ws.argtypes = [P, f32p, f32p, f32p, i32p, i32p, u8p, vp, ctypes.c_size_t, vp]
+    lib.sbsa_select_workspace_bytes.argtypes = [P]
+    lib.sbsa_select_workspace_bytes.restype = ctypes.c_size_t
     lib.sbsa_attend.argtypes = [P, vp, vp, vp, i32p, i32p, vp, vp]
     lib.sbsa_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i32p, i32p, u8p, vp]
     lib.sbsa_prefill_workspace_bytes.argtypes = [P]
@@ -136,7 +143,8 @@ def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
 def make_params(*, n_q_heads, n_kv_heads, seq_len, head_dim, block_size, dtype="bf16",
                 select_mode="topk", top_k=0, mass_threshold=0.0, rescue_tau=None,
                 gate_margin=None, group_shared=False, index_dim=0, max_blocks=None,
-                sm_scale=0.0, score_scale=0.0, backbone="mean") -> Params:
+                sm_scale=0.0, score_scale=0.0, backbone="mean", gate_quantile=None,
+                gate_rho=2) -> Params:
     p = Params()
     p.n_q_heads, p.n_kv_heads, p.seq_len = n_q_heads, n_kv_heads, seq_len
     p.head_dim, p.block_size = head_dim, block_size
@@ -148,14 +156,19 @@ def make_params(*, n_q_heads, n_kv_heads, seq_len, head_dim, block_size, dtype="
     p.mass_threshold = mass_threshold
     p.rescue = 0 if rescue_tau is None else 1
     p.rescue_tau = 0.0 if rescue_tau is None else float(rescue_tau)
-    p.gate = 0 if gate_margin is None else 1
+    if gate_margin is not None and gate_quantile is not None:
+        raise ValueError("choose one gate: gate_margin (gap) or gate_quantile (percentile)")
+    p.gate = GATE_GAP if gate_margin is not None else (
+        GATE_PERCENTILE if gate_quantile is not None else 0)
     p.gate_margin = 0.0 if gate_margin is None else float(gate_margin)
+    p.gate_quantile = 0.0 if gate_quantile is None else float(gate_quantile)
+    p.gate_rho = int(gate_rho)
     nb = (seq_len + block_size - 1) // block_size
     if max_blocks is None:
         if p.select_mode == CUMMASS or p.rescue:
             max_blocks = nb
         else:
-            budget = 2 * top_k if p.gate else top_k
+            budget = {0: top_k, GATE_GAP: 2 * top_k, GATE_PERCENTILE: p.gate_rho * top_k}[p.gate]
             max_blocks = min(budget, nb - 1) + 1
     p.max_blocks = max_blocks
     p.sm_scale = sm_scale
@@ -173,7 +186,9 @@ def params_for(w) -> Params:
                        mass_threshold=w.mass_threshold, rescue_tau=w.rescue_tau,
                        gate_margin=w.gate_margin, group_shared=w.group_shared,
                        index_dim=w.index_dim, max_blocks=w.max_blocks,
-                       backbone=getattr(w, "backbone", "mean"))
+                       backbone=getattr(w, "backbone", "mean"),
+                       gate_quantile=getattr(w, "gate_quantile", None),
+                       gate_rho=getattr(w, "gate_rho", 2))
 
 
 _TORCH_DT = {BF16: torch.bfloat16, FP32: torch.float32}
@@ -221,9 +236,11 @@ def select(p: Params, q_cent: torch.Tensor, k_cent: torch.Tensor,
     idx = torch.empty(hs, nb, p.max_blocks, device=dev, dtype=torch.int32)
     cnt = torch.empty(hs, nb, device=dev, dtype=torch.int32)
     flags = torch.empty(hs, nb, device=dev, dtype=torch.uint8) if with_flags else None
-    _check(lib.sbsa_select(ctypes.byref(p), _ptr(q_cent), _ptr(k_cent),
-                           _ptr(k_radius) if p.rescue else None, _ptr(idx), _ptr(cnt),
-                           _ptr(flags), _stream(stream)), "sbsa_select")
+    wsb = int(lib.sbsa_select_workspace_bytes(ctypes.byref(p)))
+    ws = torch.empty(wsb, device=dev, dtype=torch.uint8) if wsb else None
+    _check(lib.sbsa_select_ws(ctypes.byref(p), _ptr(q_cent), _ptr(k_cent),
+                              _ptr(k_radius) if p.rescue else None, _ptr(idx), _ptr(cnt),
+                              _ptr(flags), _ptr(ws), wsb, _stream(stream)), "sbsa_select_ws")
     return idx, cnt, flags
 
 
@@ -322,6 +339,9 @@ class Staged:
         self.idx = torch.empty(hs, nb, p.max_blocks, device=device, dtype=torch.int32)
         self.cnt = torch.empty(hs, nb, device=device, dtype=torch.int32)
         self.flags = torch.empty(hs, nb, device=device, dtype=torch.uint8)
+        self.ws_bytes = int(lib.sbsa_select_workspace_bytes(ctypes.byref(p)))
+        self.ws = (torch.empty(self.ws_bytes, device=device, dtype=torch.uint8)
+                   if self.ws_bytes else None)
         self._p = ctypes.byref(p)
 
     def pool(self, q_src, k_src, stream=None):
@@ -338,9 +358,10 @@ class Staged:
                                     None, s), "sbsa_pool_blocks")
 
     def select(self, stream=None):
-        _check(lib.sbsa_select(self._p, _ptr(self.qc), _ptr(self.kc), _ptr(self.kr),
-                               _ptr(self.idx), _ptr(self.cnt), _ptr(self.flags),
-                               _stream(stream)), "sbsa_select")
+        _check(lib.sbsa_select_ws(self._p, _ptr(self.qc), _ptr(self.kc), _ptr(self.kr),
+                                  _ptr(self.idx), _ptr(self.cnt), _ptr(self.flags),
+                                  _ptr(self.ws), self.ws_bytes, _stream(stream)),
+               "sbsa_select_ws")
 
     def attend(self, q, k, v, out, stream=None):
         _check(lib.sbsa_attend(self._p, _ptr(q), _ptr(k), _ptr(v), _ptr(self.idx),

@@ -28,6 +28,9 @@ Five workload families, one per configuration of the benchmark suite:
 * ``quest32k`` 32/8 heads, d=128, N=32768, B=128, bf16, top-16 per query head
               scored by the K-min/K-max upper bound; the RBS recipe's clustered
               keys with outliers, whose blocks the bound is designed to catch.
+* ``sigma64k`` the gate recipe at 64k (32/8 heads, B=64, top-8) with the
+              page's own gate instead of the gap test: tiles whose head-averaged
+              normalised cut margin is in the lowest 30% take the top 16.
 
 The pages behind the method (RBS-Attention, "Uncertainty-gated selection for
 block-sparse attention", MiniMax Sparse Attention) evaluate on long-context
@@ -61,6 +64,8 @@ class Workload:
     index_dim: int = 0
     seed: int = 0
     backbone: str = "mean"          # "mean" (centroids) | "minmax" (K-min/K-max bound)
+    gate_quantile: Optional[float] = None  # the page's percentile gate: q ...
+    gate_rho: int = 2                      # ... and the expansion factor rho
 
     @property
     def n_blocks(self) -> int:
@@ -85,6 +90,8 @@ class Workload:
             return self.n_blocks
         if self.gate_margin is not None:
             return min(2 * self.top_k, self.n_blocks - 1) + 1
+        if self.gate_quantile is not None:
+            return min(self.gate_rho * self.top_k, self.n_blocks - 1) + 1
         return min(self.top_k, self.n_blocks - 1) + 1
 
     def scaled(self, **kw) -> "Workload":
@@ -106,6 +113,8 @@ CONFIGS = {
                         seed=1005),
     "quest32k": Workload("quest32k", "rbs", 32, 8, 32768, 128, 128, "bf16", "topk",
                          top_k=16, seed=1006, backbone="minmax"),
+    "sigma64k": Workload("sigma64k", "gate", 32, 8, 65536, 128, 64, "bf16", "topk",
+                         top_k=8, seed=1004, gate_quantile=0.3, gate_rho=2),
 }
 
 # Reduced shapes of the same recipes, small enough for the CPU oracle to
@@ -128,6 +137,11 @@ SMALL = {
     "quest_gate_small": CONFIGS["quest32k"].scaled(name="quest_gate_small", n_q_heads=4,
                                                    n_kv_heads=2, seq_len=8192 + 50, top_k=8,
                                                    gate_margin=0.05),
+    "sigma_small": CONFIGS["sigma64k"].scaled(name="sigma_small", n_q_heads=4, n_kv_heads=2,
+                                              seq_len=8192),
+    "sigma_quest_small": CONFIGS["quest32k"].scaled(name="sigma_quest_small", n_q_heads=4,
+                                                    n_kv_heads=2, seq_len=8192 + 50, top_k=8,
+                                                    gate_quantile=0.5, gate_rho=3),
 }
 
 TORCH_DTYPE = {"bf16": torch.bfloat16, "fp32": torch.float32}

@@ -84,8 +84,10 @@ typedef struct sbsa_params {
   float mass_threshold; /* CUMMASS threshold in (0, 1]                         */
   int rescue;           /* 1: unite with the rescue branch (needs radii)       */
   float rescue_tau;     /* rescue keeps j when (q.c_j + |q| r_j)*score_scale > tau */
-  int gate;             /* 1: uncertainty gate (TOPK only)                     */
-  float gate_margin;    /* gate fires when s_(k) - s_(k+1) < margin * std(s)   */
+  int gate;             /* TOPK only. 0: none; SBSA_GATE_GAP: a row takes 2k when
+                           s_(k) - s_(k+1) < gate_margin * std(s);
+                           SBSA_GATE_PERCENTILE: the page's gate, see below    */
+  float gate_margin;    /* SBSA_GATE_GAP margin                                */
   int max_blocks;       /* list width Kmax; must hold the widest possible list:
                            TOPK min(k,NB-1)+1, gated min(2k,NB-1)+1,
                            CUMMASS or rescue NB                                */
@@ -93,7 +95,19 @@ typedef struct sbsa_params {
   float score_scale;    /* block-score scale;     0 => 1/sqrt(score dim)      */
   int backbone;         /* SBSA_BACKBONE_MEAN | SBSA_BACKBONE_MINMAX; MINMAX
                            excludes the rescue branch (which needs radii)    */
+  float gate_quantile;  /* SBSA_GATE_PERCENTILE: q in [0, 1]                  */
+  int gate_rho;         /* SBSA_GATE_PERCENTILE: fired tiles take rho*k, rho >= 1 */
 } sbsa_params;
+
+/* ---- gates ([UGS] Metodologia steps 3-5) ---- */
+#define SBSA_GATE_GAP 1        /* per row: gap at the cut below margin * std -> 2k   */
+#define SBSA_GATE_PERCENTILE 2 /* the page's gate: per row with more than k
+     candidates, sigma = (s_(k-1) - s_(k)) / (s_(0) - s_(k)) on the descending
+     0-based order (0 when s_(0) = s_(k)); per query tile, the mean of sigma over
+     the selection heads; the floor(q T) of the T eligible tiles with the
+     smallest mean (lower tile first on equal means) fire and take the top
+     rho*k in every head; max_blocks must hold min(rho*k, NB-1)+1.  Needs a
+     workspace (sbsa_select_ws or sbsa_prefill). */
 
 /*
  * sbsa_pool_blocks -- [RBS] centroid and radius of each block; [UGS] step 1
@@ -144,7 +158,24 @@ int sbsa_select(const sbsa_params* p, const float* q_cent, const float* k_cent,
                 const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags, void* stream);
 /* With p->backbone == SBSA_BACKBONE_MINMAX, k_cent is the [Hkv, NB, 2, ds]
  * table of sbsa_pool_minmax and s_j = sum_d max(q_d min_jd, q_d max_jd) *
- * score_scale; everything else is unchanged. */
+ * score_scale; everything else is unchanged.  With p->gate ==
+ * SBSA_GATE_PERCENTILE sbsa_select returns SBSA_ERR_WORKSPACE: use
+ * sbsa_select_ws. */
+
+/* Device workspace sbsa_select_ws needs (0 when no gate needs one; also 0
+ * when p is invalid). */
+size_t sbsa_select_workspace_bytes(const sbsa_params* p);
+
+/*
+ * sbsa_select_ws -- sbsa_select with a caller workspace (256-byte aligned,
+ * ws_bytes >= sbsa_select_workspace_bytes(p)) for the percentile gate's
+ * per-row margins and per-tile decisions: three launches (top-k lists and
+ * margins; the tile decisions; top-rho*k lists of the fired tiles).  The
+ * pages have no entry point; the gate is theirs.
+ */
+int sbsa_select_ws(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                   const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
+                   void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * sbsa_attend -- [RBS] sparse prefill attention; [MSA] main branch.

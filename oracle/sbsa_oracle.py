@@ -274,7 +274,8 @@ def select_row(s, i: int, *, mode: str, top_k_: int = 0, mass: float = 0.0,
 
 def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
            mass: float = 0.0, margin=None, tau=None, scale: float,
-           kv_of_sel=None, max_blocks: int, rows=None, minmax=None, sigma_gate=None):
+           kv_of_sel=None, max_blocks: int, rows=None, minmax=None, sigma_gate=None,
+           info=None):
     """Lists for every selection head hs and query block i (or the (hs, i)
     pairs in ``rows``).  ``qbar`` is [Hs, NB, d_s] and ``c``/``r`` are the key
     tables [Hkv, NB, ...]; ``kv_of_sel(hs)`` gives the kv head whose key table
@@ -305,6 +306,8 @@ def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
                 tot += cut_margin(scores(h, i), top_k_)
             sbar[i] = tot / hs_n
         fired = percentile_fire(sbar, q)
+        if info is not None:
+            info["sbar"], info["fired"] = sbar, fired
     for (h, i) in pairs:
         g = kv_of_sel(h)
         s = scores(h, i)
@@ -441,11 +444,12 @@ def prefill(q, k, v, *, block: int, mode: str, top_k_: int = 0,
     else:
         qbar = pool_queries(qs, block, group=1)
         kv_of_sel = lambda hs: hs // grp
+    info = {}
     idx, cnt, flags = select(qbar, c, r, block_count=nb, mode=mode, top_k_=top_k_,
                              mass=mass, margin=margin, tau=tau, scale=score_scale,
                              kv_of_sel=kv_of_sel, max_blocks=max_blocks,
-                             rows=sel_rows, minmax=minmax, sigma_gate=sigma_gate)
+                             rows=sel_rows, minmax=minmax, sigma_gate=sigma_gate, info=info)
     out = attend(q, k, v, idx, cnt, block=block, scale=scale,
                  group_shared=group_shared, rows=attend_rows)
     return dict(c=c, r=r, qbar=qbar, idx=idx, cnt=cnt, flags=flags, o=out,
-                minmax=minmax)
+                minmax=minmax, sbar=info.get("sbar"), fired=info.get("fired"))

@@ -18,6 +18,27 @@ import oracle as O
 BAND = 1e-5
 MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
+# A tile's head-averaged cut margin is a ratio of score differences; one fp32
+# ulp in a score near a tie moves it by far more than the score band, so the
+# percentile gate's decision is free within this absolute band of the cut.
+SIGMA_BAND = 1e-4
+
+
+def percentile_budgets(sbar: dict, fired: set, k: int, rho: int) -> dict:
+    """Budgets each tile may take under the percentile gate: rho*k when it
+    fired, k when it did not, either when its mean margin lies within
+    SIGMA_BAND of the cut between the last fired and the first kept tile."""
+    order = sorted(sbar, key=lambda i: (sbar[i], i))
+    n_fire = len(fired)
+    lo = sbar[order[n_fire - 1]] if n_fire > 0 else -math.inf
+    hi = sbar[order[n_fire]] if n_fire < len(order) else math.inf
+    out = {}
+    for i, v in sbar.items():
+        b = {rho * k} if i in fired else {k}
+        if abs(v - lo) <= SIGMA_BAND or abs(v - hi) <= SIGMA_BAND:
+            b = {k, rho * k}
+        out[i] = b
+    return out
 
 
 def band(x: float) -> float:
@@ -28,7 +49,7 @@ def near(a: float, b: float) -> bool:
     return abs(a - b) <= band(max(abs(a), abs(b)))
 
 
-def _base_alternatives(s, i, w):
+def _base_alternatives(s, i, w, budgets_i=None):
     """Base-branch sets the oracle's decisions allow within the tie band,
     as (must_have, may_have, sizes) triples."""
     s64 = np.asarray(s, dtype=np.float64)
@@ -37,7 +58,9 @@ def _base_alternatives(s, i, w):
     alts = []
     if w.select_mode == "topk":
         budgets = [w.top_k]
-        if w.gate_margin is not None and n > w.top_k:
+        if budgets_i is not None:
+            budgets = sorted(budgets_i)
+        elif w.gate_margin is not None and n > w.top_k:
             fired, gap, thr = O.gate(s, w.top_k, w.gate_margin)
             if abs(gap - thr) <= band(thr):
                 budgets = [w.top_k, 2 * w.top_k]
@@ -70,7 +93,7 @@ def _base_alternatives(s, i, w):
     return alts
 
 
-def row_matches(gpu_ids, s, ub, i, w):
+def row_matches(gpu_ids, s, ub, i, w, budgets_i=None):
     """True when the GPU list of query block i is allowed by the oracle's
     decisions (exact or within the tie band)."""
     g = set(int(x) for x in gpu_ids)
@@ -92,7 +115,7 @@ def row_matches(gpu_ids, s, ub, i, w):
         return False
     r_range = rescue_must | rescue_may
     x = body - r_range                      # blocks only the base branch can explain
-    for must, may, sizes in _base_alternatives(s, i, w):
+    for must, may, sizes in _base_alternatives(s, i, w, budgets_i):
         if not must <= body or not x <= (must | may):
             continue
         lo = len(must | x)
@@ -103,10 +126,12 @@ def row_matches(gpu_ids, s, ub, i, w):
 
 
 def compare_lists(gpu_idx, gpu_cnt, oracle_idx, oracle_cnt, rows, qbar, c, r, w, kv_of_sel,
-                  minmax=None):
+                  minmax=None, budgets=None):
     """Returns (exact, tie) counts over ``rows``; raises AssertionError on a
     difference the tie band does not explain.  ``minmax`` = (kmin, kmax)
-    selects the upper-bound backbone's scores instead of the centroids'."""
+    selects the upper-bound backbone's scores instead of the centroids';
+    ``budgets`` (tile -> allowed top-k budgets) carries the percentile gate's
+    decisions."""
     exact = tie = 0
     scale = 1.0 / math.sqrt(w.score_dim)
     for (hs, i) in rows:
@@ -121,7 +146,7 @@ def compare_lists(gpu_idx, gpu_cnt, oracle_idx, oracle_cnt, rows, qbar, c, r, w,
         else:
             s = O.block_bounds_minmax(qbar[hs, i], minmax[0][g], minmax[1][g], i, scale)
         ub = O.rescue_bounds(qbar[hs, i], c[g], r[g], i, scale) if w.rescue_tau is not None else None
-        if not row_matches(gi, s, ub, i, w):
+        if not row_matches(gi, s, ub, i, w, None if budgets is None else budgets.get(i)):
             raise AssertionError(f"row (head {hs}, block {i}): gpu {gi} vs oracle {oi}")
         tie += 1
     return exact, tie

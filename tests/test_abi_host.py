@@ -55,7 +55,8 @@ int main(void) {
   printf("size %zu\n", sizeof(sbsa_params));
   F(n_q_heads) F(n_kv_heads) F(seq_len) F(head_dim) F(block_size) F(dtype) F(select_mode)
   F(group_shared) F(index_dim) F(top_k) F(mass_threshold) F(rescue) F(rescue_tau) F(gate)
-  F(gate_margin) F(max_blocks) F(sm_scale) F(score_scale) F(backbone)
+  F(gate_margin) F(max_blocks) F(sm_scale) F(score_scale) F(backbone) F(gate_quantile)
+  F(gate_rho)
   return 0;
 }
 '''
@@ -111,6 +112,10 @@ def _attend(sb, p):
     (dict(select_mode="cummass", mass_threshold=0.9, max_blocks=5), 1),  # needs NB
     (dict(sm_scale=-1.0), 1),
     (dict(backbone=2), 1),                       # no such backbone
+    (dict(gate_quantile=1.5), 1),                # q outside [0, 1]
+    (dict(gate_quantile=0.3, gate_rho=0), 1),
+    (dict(gate_quantile=0.3, gate_rho=3, max_blocks=7), 1),   # needs min(rho*k, NB-1)+1 = 8
+    (dict(select_mode="cummass", mass_threshold=0.9, gate_quantile=0.3), 1),
     (dict(select_mode="cummass", mass_threshold=0.9, rescue_tau=5.0, backbone="minmax"), 1),
 ])
 def test_invalid_parameters_are_rejected_before_launch(sb, mutate, code):
@@ -162,6 +167,22 @@ def test_minmax_backbone_doubles_the_key_table_in_the_workspace(sb):
         return (x + 255) // 256 * 256
     extra = r256(2 * 2 * nb * 128 * 4) - r256(2 * nb * 128 * 4)
     assert sb.workspace_bytes(mm) == sb.workspace_bytes(mean) + extra
+
+
+def test_percentile_gate_needs_a_workspace(sb):
+    p = _valid(sb, gate_quantile=0.3, gate_rho=2, seq_len=4096)
+    nb = p.n_blocks
+    need = sb.lib.sbsa_select_workspace_bytes(ctypes.byref(p))
+    assert need == (4 * nb * 8 + 255) // 256 * 256 + (nb + 255) // 256 * 256
+    assert sb.lib.sbsa_select_workspace_bytes(ctypes.byref(_valid(sb))) == 0
+    assert _select(sb, p) == 3                   # the plain entry point has no workspace
+    ws = sb.lib.sbsa_select_ws
+    assert ws(ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, None, FAKE, need - 1, None) == 3
+    assert ws(ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, None,
+              ctypes.c_void_p((1 << 20) + 64), need, None) == 3
+    # the prefill workspace grows by the same scratch
+    plain = sb.workspace_bytes(_valid(sb, seq_len=4096, max_blocks=p.max_blocks))
+    assert sb.workspace_bytes(p) == plain + need
 
 
 def test_fp32_attention_is_limited_to_d64_b64(sb):

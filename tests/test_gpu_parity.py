@@ -15,7 +15,7 @@ from block_sparse_attention_sbsa_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 SMALL_NAMES = ["tiny", "gqa_small", "rbs_small", "gate_small", "msa_small", "quest_small",
-               "quest_gate_small"]
+               "quest_gate_small", "sigma_small", "sigma_quest_small"]
 
 
 @pytest.fixture(scope="module")
@@ -26,11 +26,24 @@ def sb(cuda):
     return sbsa
 
 
+def _sigma_gate(w):
+    # q as the float32 the kernels receive
+    return None if w.gate_quantile is None else (float(np.float32(w.gate_quantile)), w.gate_rho)
+
+
+def _budgets(w, ref):
+    """Tile -> allowed budgets under the percentile gate (None otherwise)."""
+    if w.gate_quantile is None:
+        return None
+    return PT.percentile_budgets(ref["sbar"], ref["fired"], w.top_k, w.gate_rho)
+
+
 def _oracle_prefill(w, data, **kw):
     return O.prefill(data["q"], data["k"], data["v"], block=w.block_size, mode=w.select_mode,
                      top_k_=w.top_k, mass=w.mass_threshold, margin=w.gate_margin,
                      tau=w.rescue_tau, group_shared=w.group_shared, q_idx=data["q_idx"],
-                     k_idx=data["k_idx"], max_blocks=w.max_blocks, backbone=w.backbone, **kw)
+                     k_idx=data["k_idx"], max_blocks=w.max_blocks, backbone=w.backbone,
+                     sigma_gate=_sigma_gate(w), **kw)
 
 
 @functools.lru_cache(maxsize=None)
@@ -88,7 +101,8 @@ def test_select_on_oracle_tables(sb, name):
     idx, cnt, flags = sb.select(p, qc, kc, kr if w.rescue_tau is not None else None)
     idx, cnt, flags = idx.cpu().numpy(), cnt.cpu().numpy(), flags.cpu().numpy()
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
-                                  ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"])
+                                  ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"],
+                                  budgets=_budgets(w, ref))
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # padding and flags
     for hs in range(w.n_sel_heads):
@@ -124,7 +138,8 @@ def test_prefill_end_to_end(sb, name):
     assert sb.get_status() == sb.OK
     idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
-                                  ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"])
+                                  ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"],
+                                  budgets=_budgets(w, ref))
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # outputs on query rows whose lists match the oracle exactly
     o = o.float().cpu().numpy()
@@ -150,7 +165,7 @@ def test_gate_fires_on_the_planted_rows(sb):
 
 # ------------------------------------------------------------- full sizes
 
-FULL = ["gqa32k", "rbs128k", "gate64k", "msa512k", "quest32k"]
+FULL = ["gqa32k", "rbs128k", "gate64k", "msa512k", "quest32k", "sigma64k"]
 
 
 def _sample_blocks(w, meta, count):
@@ -184,18 +199,23 @@ def test_full_size_sampled(sb, name):
     mmx = O.pool_keys_minmax(ks, w.block_size) if w.backbone == "minmax" else None
     nb = w.n_blocks
     qrows = torch.cat([qs[:, i * w.block_size:(i + 1) * w.block_size] for i in blocks], dim=1).cpu()
-    # pooled queries of the sampled blocks only
+    # pooled queries of the sampled blocks only (of every block when the
+    # percentile gate needs every tile's margin)
     qbar = np.zeros((w.n_sel_heads, nb, w.score_dim))
     grp = w.group if w.group_shared else 1
+    if w.gate_quantile is not None:
+        qbar = O.pool_queries(qs.cpu(), w.block_size, group=grp)
     for bi, i in enumerate(blocks):
         rows = qrows[:, bi * w.block_size:(bi + 1) * w.block_size]
         qb = O.pool_queries(rows, w.block_size, group=grp)
         qbar[:, i] = qb[:, 0]
     sel_rows = [(hs, i) for hs in range(w.n_sel_heads) for i in blocks]
+    info = {}
     idx, cnt, flags = O.select(qbar, c, r, block_count=nb, mode=w.select_mode, top_k_=w.top_k,
                                mass=w.mass_threshold, margin=w.gate_margin, tau=w.rescue_tau,
                                scale=1.0 / math.sqrt(w.score_dim), kv_of_sel=_kv_of_sel(w),
-                               max_blocks=w.max_blocks, rows=sel_rows, minmax=mmx)
+                               max_blocks=w.max_blocks, rows=sel_rows, minmax=mmx,
+                               sigma_gate=_sigma_gate(w), info=info)
     gidx = call.idx[:, blocks].cpu().numpy()
     gcnt = call.cnt[:, blocks].cpu().numpy()
     gi_full = np.full((w.n_sel_heads, nb, w.max_blocks), -1, dtype=np.int32)
@@ -203,7 +223,7 @@ def test_full_size_sampled(sb, name):
     gi_full[:, blocks] = gidx
     gc_full[:, blocks] = gcnt
     exact, tie = PT.compare_lists(gi_full, gc_full, idx, cnt, sel_rows, qbar, c, r, w,
-                                  _kv_of_sel(w), minmax=mmx)
+                                  _kv_of_sel(w), minmax=mmx, budgets=_budgets(w, info))
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # outputs of the sampled blocks whose lists match (all query heads; two
     # per group for the 64-head workload); keys/values converted once per
