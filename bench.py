@@ -6,8 +6,11 @@ mass 0.9 united with the radius rescue branch).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sbsa|reference]
 
-One process per GPU (torchrun for N > 1).  Every rank runs its own
-independent sequence (weak scaling, no collective on the data path); the
+One process per GPU (torchrun for N > 1).  By default every rank runs its
+own independent sequence (weak scaling); with --shard heads the ranks split
+one sequence by kv head, each prefilling its kv heads and their query heads
+(strong scaling).  Neither mode has a collective on the data path: the
+selection and the attention of a kv head need nothing from another.  The
 reported time is the maximum over ranks.  Rank 0 prints one JSON line.
 `--impl reference` times the CPU oracle on a bounded sample of the same
 workload instead.
@@ -99,6 +102,9 @@ def parse_args():
     ap.add_argument("--cpu-blocks", type=int, default=6,
                     help="query blocks (all heads) in the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
+                    help="N > 1: independent sequences per rank (weak scaling) or one "
+                         "sequence split by kv head (strong scaling)")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override the workload length (small cases for profiling)")
     return ap.parse_args()
@@ -309,6 +315,35 @@ def rank_workload(base, rank: int):
     return base.scaled(seed=base.seed + 1000 * rank)
 
 
+def head_shard(n_kv_heads: int, rank: int, world: int):
+    """Contiguous kv-head range [g0, g1) of a rank when one sequence is split
+    by kv head: as even as possible, the first ranks take one more."""
+    if world > n_kv_heads:
+        raise ValueError(f"{world} ranks cannot split {n_kv_heads} kv heads")
+    base, rem = divmod(n_kv_heads, world)
+    g0 = rank * base + min(rank, rem)
+    return g0, g0 + base + (1 if rank < rem else 0)
+
+
+def shard_workload(w, rank: int, world: int):
+    """The sub-problem of one rank under head sharding: its kv heads and the
+    query heads that read them, same sequence and seed."""
+    g0, g1 = head_shard(w.n_kv_heads, rank, world)
+    return w.scaled(n_q_heads=(g1 - g0) * w.group, n_kv_heads=g1 - g0), (g0, g1)
+
+
+def shard_tensors(data: dict, w_full, g0: int, g1: int) -> dict:
+    """Head slices of a generated workload (head-major layout: contiguous)."""
+    grp = w_full.group
+    out = dict(data)
+    out["q"] = data["q"][g0 * grp:g1 * grp]
+    out["k"], out["v"] = data["k"][g0:g1], data["v"][g0:g1]
+    if data.get("q_idx") is not None:
+        out["q_idx"] = data["q_idx"][g0 * grp:g1 * grp]
+        out["k_idx"] = data["k_idx"][g0:g1]
+    return out
+
+
 def reduce_max(values, device="cpu"):
     """Element-wise maximum over ranks (identity on one process)."""
     import torch
@@ -342,8 +377,19 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300))
 
-    w = rank_workload(pick_workload(args), rank)
-    data = W.generate(w, "cuda")
+    heads = args.shard == "heads" and world > 1
+    if heads:
+        # every rank draws the same sequence and keeps its kv heads
+        w_full = pick_workload(args)
+        if w_full.gate_quantile is not None:
+            raise SystemExit("--shard heads: the percentile gate averages its margins over all "
+                             "heads of a tile, which would need an all-reduce between its "
+                             "passes; shard by sequences instead")
+        w, (g0, g1) = shard_workload(w_full, rank, world)
+        data = shard_tensors(W.generate(w_full, "cuda"), w_full, g0, g1)
+    else:
+        w_full = w = rank_workload(pick_workload(args), rank)
+        data = W.generate(w, "cuda")
     p = sbsa.params_for(w)
     st = sbsa.Staged(p)
     q, k, v = data["q"], data["k"], data["v"]
@@ -374,7 +420,8 @@ def main():
     pairs = sbsa.attended_pairs(p, st.cnt)
     attend_flops = 4.0 * w.head_dim * pairs
     mean_cnt = float(st.cnt.float().mean())
-    sel_stats = selection_stats(w, p, st, data.get("meta", {}))
+    # planted needles are indexed by the full problem's kv heads
+    sel_stats = selection_stats(w, p, st, {} if heads else data.get("meta", {}))
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -440,7 +487,7 @@ def main():
         return 0
 
     peaks, src = load_peaks()
-    value = weak_throughput(w.seq_len, world, args.steps, elapsed_ms)
+    value = weak_throughput(w.seq_len, 1 if heads else world, args.steps, elapsed_ms)
     ms_per_step = elapsed_ms / args.steps
     att_tflops = attend_flops / (att_ms / 1000.0) / 1e12
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -456,9 +503,12 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+        "scaling": "strong" if heads else "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "fp32",
         "data": "synthetic (seeded generator, RBS-style clustered keys with outliers)",
-        "config": workload_config(w),
+        "config": dict(workload_config(w_full),
+                       parallelism=(f"kv heads split over {world} GPUs" if heads else
+                                    f"{world} independent sequence(s), one per GPU")),
         "attended_tflops": att_tflops,
         "roofline": {
             "bound": "tensor", "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",

@@ -47,3 +47,75 @@ def test_two_ranks_take_the_slowest_time_and_distinct_sequences():
 def test_single_process_reduce_is_identity():
     import bench
     assert bench.reduce_max([1.5, 2.5]) == [1.5, 2.5]
+
+
+# ------------------------------------------------ head-sharded prefill
+
+@pytest.mark.parametrize("hkv,world", [(8, 1), (8, 2), (8, 3), (8, 8), (2, 2), (1, 1)])
+def test_head_shards_partition_the_kv_heads(hkv, world):
+    import bench
+    ranges = [bench.head_shard(hkv, r, world) for r in range(world)]
+    assert ranges[0][0] == 0 and ranges[-1][1] == hkv
+    for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
+        assert a1 == b0
+    sizes = [g1 - g0 for g0, g1 in ranges]
+    assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+
+
+def test_more_ranks_than_kv_heads_is_refused():
+    import bench
+    with pytest.raises(ValueError):
+        bench.head_shard(2, 0, 3)
+
+
+@pytest.mark.parametrize("name", ["gqa_small", "msa_small", "quest_gate_small"])
+def test_the_method_decomposes_by_kv_head(name):
+    """Head sharding is exact: the oracle on each rank's kv heads (and the
+    query heads reading them) reproduces the full problem's lists and output
+    rows of those heads."""
+    import numpy as np
+    import bench
+    import oracle as O
+    from block_sparse_attention_sbsa_b200 import workloads as W
+    w = W.SMALL[name].scaled(seq_len=1024 + 37)
+    data = W.generate(w, "cpu")
+
+    def run(wk, d):
+        return O.prefill(d["q"], d["k"], d["v"], block=wk.block_size, mode=wk.select_mode,
+                         top_k_=wk.top_k, mass=wk.mass_threshold, margin=wk.gate_margin,
+                         tau=wk.rescue_tau, group_shared=wk.group_shared, q_idx=d["q_idx"],
+                         k_idx=d["k_idx"], max_blocks=wk.max_blocks, backbone=wk.backbone)
+    full = run(w, data)
+    for rank in range(2):
+        ws, (g0, g1) = bench.shard_workload(w, rank, 2)
+        part = run(ws, bench.shard_tensors(data, w, g0, g1))
+        hs0, hs1 = (g0, g1) if w.group_shared else (g0 * w.group, g1 * w.group)
+        assert np.array_equal(part["idx"], full["idx"][hs0:hs1])
+        assert np.array_equal(part["o"], full["o"][g0 * w.group:g1 * w.group])
+
+
+def _shard_worker(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    from block_sparse_attention_sbsa_b200 import workloads as W
+    ws, (g0, g1) = bench.shard_workload(W.CONFIGS["rbs128k"], rank, world)
+    got = bench.reduce_max([float(ws.n_kv_heads), float(g1)])
+    out[rank] = (g0, g1, ws.n_q_heads, got)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_ranks_split_one_sequence_by_kv_head():
+    world, port = 2, _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
+    assert (out[0][0], out[0][1]) == (0, 4) and (out[1][0], out[1][1]) == (4, 8)
+    assert out[0][2] == out[1][2] == 16
+    assert out[0][3] == out[1][3] == [4.0, 8.0]
+    import bench
+    # one sequence of 131072 tokens, 3 steps, slowest rank 30 ms
+    assert bench.weak_throughput(131072, 1, 3, 30.0) == pytest.approx(131072 * 3 / 0.03)
