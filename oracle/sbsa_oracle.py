@@ -43,6 +43,12 @@ candidates and keeps the shortest prefix of the ranked order whose mass
 reaches the threshold; the rescue test is (q.c + |q| r) * scale > tau.
 The K-min/K-max backbone bounds q.k over the block's keys coordinate by
 coordinate: sum_d max(q_d * min_d, q_d * max_d), scaled like the mean score.
+Row-max tile scores (Metodologia step 2: the tile score is the largest
+score among the tile's query rows): s_ij = max_t (q_t . c_j) * scale over
+the rows t of query block i (and, in group mode, over the heads of the
+group); the kernels take this contraction on bf16 tensor cores, so the
+decision precision is theirs: centroids rounded to bf16, products exact,
+the sum and the maximum in float64, the result rounded to float32.
 The page's own gate (Metodologia steps 3-5): the normalised cut margin
 sigma = (s_(k-1) - s_(k)) / (s_(0) - s_(k)) on the descending 0-based order
 (0 when s_(0) = s_(k)), defined for rows with more than k candidates; its
@@ -164,6 +170,25 @@ def block_bounds_minmax(qbar_i, kmin_g, kmax_g, i: int, scale: float):
     return (np.maximum(lo, hi).sum(axis=1) * scale).astype(np.float32)
 
 
+def bf16_round(x) -> np.ndarray:
+    """Round-to-nearest-even to bfloat16, returned as float64."""
+    f = np.asarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def block_scores_rowmax(q_rows, c_g, i: int, scale: float):
+    """Tile score of query block i against candidates j < i: the largest
+    q_t . bf16(c_j) over the tile's query rows t (all rows given, e.g. the
+    rows of every head of a group), times scale, rounded to float32."""
+    q = _f64(q_rows)
+    c = bf16_round(c_g[:i])
+    if i == 0:
+        return np.zeros(0, dtype=np.float32)
+    return ((q @ c.T).max(axis=0) * scale).astype(np.float32)
+
+
 def rescue_bounds(qbar_i, c_g, r_g, i: int, scale: float):
     """Upper bound of q.k over block j when k lies within r_j of c_j
     (Cauchy-Schwarz): (qbar . c_j + |qbar| r_j) * scale, rounded to float32."""
@@ -275,7 +300,7 @@ def select_row(s, i: int, *, mode: str, top_k_: int = 0, mass: float = 0.0,
 def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
            mass: float = 0.0, margin=None, tau=None, scale: float,
            kv_of_sel=None, max_blocks: int, rows=None, minmax=None, sigma_gate=None,
-           info=None):
+           info=None, row_scores=None):
     """Lists for every selection head hs and query block i (or the (hs, i)
     pairs in ``rows``).  ``qbar`` is [Hs, NB, d_s] and ``c``/``r`` are the key
     tables [Hkv, NB, ...]; ``kv_of_sel(hs)`` gives the kv head whose key table
@@ -290,6 +315,8 @@ def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
 
     def scores(h, i):
         g = kv_of_sel(h)
+        if row_scores is not None:
+            return row_scores(h, i)
         if minmax is None:
             return block_scores(qbar[h, i], c[g], i, scale)
         return block_bounds_minmax(qbar[h, i], minmax[0][g], minmax[1][g], i, scale)
@@ -413,7 +440,7 @@ def prefill(q, k, v, *, block: int, mode: str, top_k_: int = 0,
             mass: float = 0.0, margin=None, tau=None, group_shared: bool = False,
             q_idx=None, k_idx=None, max_blocks: int, scale=None,
             score_scale=None, sel_rows=None, attend_rows=None, backbone: str = "mean",
-            sigma_gate=None):
+            sigma_gate=None, tile_score: str = "mean"):
     """Selection tables and lists from the index tensors (q_idx/k_idx when
     given, else q/k), then attention over the lists.  ``sel_rows`` restricts
     selection to (hs, i) pairs, ``attend_rows`` restricts attention to
@@ -444,11 +471,25 @@ def prefill(q, k, v, *, block: int, mode: str, top_k_: int = 0,
     else:
         qbar = pool_queries(qs, block, group=1)
         kv_of_sel = lambda hs: hs // grp
+    row_scores = None
+    if tile_score == "rowmax":
+        if backbone != "mean" or tau is not None:
+            raise ValueError("row-max tile scores use the centroids, without the rescue branch")
+
+        def row_scores(h, i):
+            heads = range(h * grp, (h + 1) * grp) if group_shared else [h]
+            rows = np.concatenate([_f64(qs[hh, i * block:min(n, (i + 1) * block)])
+                                   for hh in heads])
+            return block_scores_rowmax(rows, c[h if group_shared else h // grp], i,
+                                       score_scale)
+    elif tile_score != "mean":
+        raise ValueError(tile_score)
     info = {}
     idx, cnt, flags = select(qbar, c, r, block_count=nb, mode=mode, top_k_=top_k_,
                              mass=mass, margin=margin, tau=tau, scale=score_scale,
                              kv_of_sel=kv_of_sel, max_blocks=max_blocks,
-                             rows=sel_rows, minmax=minmax, sigma_gate=sigma_gate, info=info)
+                             rows=sel_rows, minmax=minmax, sigma_gate=sigma_gate, info=info,
+                             row_scores=row_scores)
     out = attend(q, k, v, idx, cnt, block=block, scale=scale,
                  group_shared=group_shared, rows=attend_rows)
     return dict(c=c, r=r, qbar=qbar, idx=idx, cnt=cnt, flags=flags, o=out,

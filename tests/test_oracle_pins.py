@@ -532,3 +532,54 @@ def test_percentile_gate_fires_the_floor_q_t_most_ambiguous_tiles(q):
 
 def test_percentile_gate_breaks_equal_margins_by_lower_tile():
     assert O.percentile_fire({5: 0.2, 3: 0.2, 9: 0.1, 7: 0.9}, 0.5) == {9, 3}
+
+
+# --------------------------------------------------------------------------
+# Row-max tile scores (uncertainty-gated page, Metodologia step 2: the tile
+# score is the largest score among the tile's query rows)
+# --------------------------------------------------------------------------
+
+def test_bf16_rounding_is_round_to_nearest_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -7, -2.0 - 2 ** -7],
+                 dtype=np.float32)
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: even (1); 1 + 3*2^-8 -> 1 + 2^-6;
+    # -2 - 2^-7 is halfway between -2 and -2 - 2^-6: even (-2)
+    assert O.bf16_round(x).tolist() == [1.0, 1.0, 1.0 + 2 ** -6, 1.0 + 2 ** -7, -2.0]
+    assert np.array_equal(O.bf16_round(x), torch.tensor(x).bfloat16().double().numpy())
+
+
+def test_rowmax_of_identical_rows_is_the_pooled_score_and_dominates_it_otherwise():
+    rng = np.random.default_rng(41)
+    c = rng.standard_normal((6, 16))
+    row = rng.standard_normal(16)
+    same = np.tile(row, (32, 1))
+    got = O.block_scores_rowmax(same, c, 6, 0.25)
+    want = (O.bf16_round(c) @ row * 0.25).astype(np.float32)
+    assert np.array_equal(got, want)
+    rows = rng.standard_normal((32, 16))
+    mx = O.block_scores_rowmax(rows, c, 6, 0.25).astype(np.float64)
+    mean = O.bf16_round(c) @ rows.mean(axis=0) * 0.25
+    assert (mx >= mean - 1e-6).all()
+    # the order of the rows does not matter
+    assert np.array_equal(O.block_scores_rowmax(rows[::-1], c, 6, 0.25), mx.astype(np.float32))
+
+
+@pytest.mark.parametrize("group_shared", [False, True])
+def test_rowmax_finds_the_block_one_query_row_points_at(group_shared):
+    """One query row of the last tile (of one head) points at block 2; the
+    mean over the tile's rows hides it, the row maximum does not."""
+    rng = np.random.default_rng(42)
+    hq, hk, n, b, d = 2, 1, 8 * 32, 32, 16
+    q = rng.standard_normal((hq, n, d)) * 0.1
+    k = rng.standard_normal((hk, n, d)) * 0.1
+    v = rng.standard_normal((hk, n, d))
+    k[0, 2 * b:3 * b, 4] += 1.5                  # block 2: centroid along e_4
+    k[0, 5 * b:6 * b, 3] += 5.0                  # block 5: along e_3
+    q[:, 7 * b:, 3] += 0.5                       # every row of the last tile leans along e_3 ...
+    q[1, 7 * b + 4, 4] = 40.0                    # ... one row of head 1 points along e_4
+    common = dict(block=b, mode="topk", top_k_=1, max_blocks=2, group_shared=group_shared)
+    mean = O.prefill(q, k, v, tile_score="mean", **common)
+    rowmax = O.prefill(q, k, v, tile_score="rowmax", **common)
+    hs = 0 if group_shared else 1
+    assert rowmax["idx"][hs, 7, :2].tolist() == [2, 7]
+    assert mean["idx"][hs, 7, :2].tolist() != [2, 7]
