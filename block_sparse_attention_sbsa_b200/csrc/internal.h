@@ -4,6 +4,7 @@
 #include <cstdint>
 
 #include "sbsa.h"
+#include <cuda_bf16.h>
 
 namespace sbsa {
 
@@ -43,6 +44,7 @@ struct SelectArgs {
   int rho;
   double* sigma;        // [Hs, NB] cut margins (NaN: no cut), written by pass 1
   const uint8_t* fire;  // [NB] 1 for fired tiles, read by pass 2
+  const float* scores;  // [Hs, NB, NB] precomputed tile scores (row-max), or nullptr
   int top_k;
   float mass;
   int gate;
@@ -59,6 +61,20 @@ cudaError_t launch_gate_tiles(const double* sigma, uint8_t* fire, int n_sel_head
                               int top_k, float quantile, cudaStream_t stream);
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+
+// Row-max tile scores: the fp32 centroids are converted to bf16 into c_bf16,
+// then scores[hs, i, j] = max over the tile's query rows (and the group's
+// heads in group mode) of q_t . c_j * scale, for j < i.
+struct RowmaxArgs {
+  const void* q;         // [Hq, N, ds] bf16 (Q, or Q_idx in index mode)
+  const float* c_f32;    // [Hkv, NB, ds]
+  __nv_bfloat16* c_bf16; // [Hkv, NB, ds] scratch
+  float* scores;         // [Hs, NB, NB]
+  int hq, hkv, n, nb, ds, group_shared;
+  float scale;
+  int* status;
+};
+cudaError_t launch_rowmax(const RowmaxArgs& a, cudaStream_t stream);
 
 struct AttendArgs {
   const void* q;

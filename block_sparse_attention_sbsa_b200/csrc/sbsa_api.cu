@@ -70,6 +70,11 @@ int validate(const sbsa_params* p, Derived* d) {
   if (p->backbone != SBSA_BACKBONE_MEAN && p->backbone != SBSA_BACKBONE_MINMAX)
     return SBSA_ERR_INVALID_ARG;
   if (p->backbone == SBSA_BACKBONE_MINMAX && p->rescue) return SBSA_ERR_INVALID_ARG;
+  if (p->tile_score != SBSA_TILE_MEAN && p->tile_score != SBSA_TILE_ROWMAX)
+    return SBSA_ERR_INVALID_ARG;
+  if (p->tile_score == SBSA_TILE_ROWMAX &&
+      (p->backbone != SBSA_BACKBONE_MEAN || p->rescue || p->dtype != SBSA_BF16))
+    return SBSA_ERR_INVALID_ARG;
   if (!(p->sm_scale >= 0.f) || !std::isfinite(p->sm_scale)) return SBSA_ERR_INVALID_ARG;
   if (!(p->score_scale >= 0.f) || !std::isfinite(p->score_scale)) return SBSA_ERR_INVALID_ARG;
   Derived o;
@@ -104,8 +109,19 @@ int attend_supported(const sbsa_params* p) {
 }
 
 struct WsLayout {
-  size_t qc, kc, kr, idx, cnt, flags, sigma, fire, total;
+  size_t qc, kc, kr, idx, cnt, flags, sigma, fire, cbf, scores, total;
 };
+
+// Scratch of the row-max tile scores: the bf16 centroids and the score table.
+size_t rowmax_scratch(const sbsa_params* p, const Derived& d, size_t off, size_t* cbf,
+                      size_t* scores) {
+  const bool on = p->tile_score == SBSA_TILE_ROWMAX;
+  *cbf = off;
+  if (on) off = round_up(off + (size_t)p->n_kv_heads * d.nb * d.ds * 2, 256);
+  *scores = off;
+  if (on) off = round_up(off + (size_t)d.hs * d.nb * d.nb * 4, 256);
+  return off;
+}
 
 // Scratch of the percentile gate: per-row margins (double) and per-tile
 // decisions, placed from offset `off`.
@@ -135,6 +151,7 @@ WsLayout layout(const sbsa_params* p, const Derived& d, bool lists) {
   w.flags = off;
   off = round_up(off + (lists ? (size_t)d.hs * d.nb : 0), 256);
   off = gate_scratch(p, d, off, &w.sigma, &w.fire);
+  off = rowmax_scratch(p, d, off, &w.cbf, &w.scores);
   w.total = off;
   return w;
 }
@@ -216,7 +233,7 @@ using namespace sbsa;
 
 extern "C" {
 
-int sbsa_version(void) { return 102; }
+int sbsa_version(void) { return 103; }
 
 const char* sbsa_status_string(int code) {
   switch (code) {
@@ -280,6 +297,65 @@ size_t sbsa_select_workspace_bytes(const sbsa_params* p) {
   if (validate(p, &d) != SBSA_OK) return 0;
   size_t sigma, fire;
   return gate_scratch(p, d, 0, &sigma, &fire);
+}
+
+size_t sbsa_score_rowmax_workspace_bytes(const sbsa_params* p) {
+  Derived d;
+  if (validate(p, &d) != SBSA_OK || p->tile_score != SBSA_TILE_ROWMAX) return 0;
+  return round_up((size_t)p->n_kv_heads * d.nb * d.ds * 2, 256);
+}
+
+namespace {
+RowmaxArgs rowmax_args(const sbsa_params* p, const Derived& d, const void* q_src,
+                       const float* k_cent, void* c_bf16, float* scores) {
+  RowmaxArgs a{};
+  a.q = q_src;
+  a.c_f32 = k_cent;
+  a.c_bf16 = static_cast<__nv_bfloat16*>(c_bf16);
+  a.scores = scores;
+  a.hq = p->n_q_heads;
+  a.hkv = p->n_kv_heads;
+  a.n = p->seq_len;
+  a.nb = d.nb;
+  a.ds = d.ds;
+  a.group_shared = p->group_shared ? 1 : 0;
+  a.scale = d.score_scale;
+  a.status = device_status_ptr();
+  return a;
+}
+}  // namespace
+
+int sbsa_score_rowmax(const sbsa_params* p, const void* q_src, const float* k_cent,
+                      float* scores, void* workspace, size_t ws_bytes, void* stream) {
+  Derived d;
+  int rc = validate(p, &d);
+  if (rc) return rc;
+  if (p->tile_score != SBSA_TILE_ROWMAX) return SBSA_ERR_UNSUPPORTED;
+  if (!q_src || !k_cent || !scores) return SBSA_ERR_INVALID_ARG;
+  if (!aligned16(q_src) || !aligned16(k_cent) || !aligned16(scores)) return SBSA_ERR_INVALID_ARG;
+  const size_t need = sbsa_score_rowmax_workspace_bytes(p);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < need)
+    return SBSA_ERR_WORKSPACE;
+  return cuda_code(launch_rowmax(rowmax_args(p, d, q_src, k_cent, workspace, scores),
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+int sbsa_select_scores(const sbsa_params* p, const float* scores, int32_t* idx, int32_t* cnt,
+                       uint8_t* flags, void* workspace, size_t ws_bytes, void* stream) {
+  Derived d;
+  int rc = validate(p, &d);
+  if (rc) return rc;
+  if (!scores || !idx || !cnt) return SBSA_ERR_INVALID_ARG;
+  if (p->rescue) return SBSA_ERR_INVALID_ARG;  // the rescue bound needs the tables
+  size_t sigma, fire;
+  const size_t need = gate_scratch(p, d, 0, &sigma, &fire);
+  if (need && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+               ws_bytes < need))
+    return SBSA_ERR_WORKSPACE;
+  SelectArgs a = select_args(p, d, nullptr, nullptr, nullptr, idx, cnt, flags);
+  a.scores = scores;
+  return run_select(p, d, a, static_cast<unsigned char*>(workspace), sigma, fire,
+                    static_cast<cudaStream_t>(stream));
 }
 
 int sbsa_select_ws(const sbsa_params* p, const float* q_cent, const float* k_cent,
@@ -355,9 +431,19 @@ int sbsa_prefill(const sbsa_params* p, const void* q, const void* k, const void*
       {xs_k, p->n_kv_heads, 1, minmax ? nullptr : kc, kr, minmax ? kc : nullptr},
       {xs_q, p->n_q_heads, p->group_shared ? d.group : 1, qc, nullptr, nullptr},
   };
-  rc = cuda_code(launch_pool(p->dtype, d.ds, p->seq_len, p->block_size, jobs, 2, s));
+  // row-max tile scores read the query rows themselves: no pooled queries
+  const bool rowmax = p->tile_score == SBSA_TILE_ROWMAX;
+  rc = cuda_code(launch_pool(p->dtype, d.ds, p->seq_len, p->block_size, jobs, rowmax ? 1 : 2, s));
   if (rc) return rc;
-  rc = run_select(p, d, select_args(p, d, qc, kc, kr, idx, cnt, flags), ws, w.sigma, w.fire, s);
+  SelectArgs sa = select_args(p, d, qc, kc, kr, idx, cnt, flags);
+  if (p->tile_score == SBSA_TILE_ROWMAX) {
+    float* scores = reinterpret_cast<float*>(ws + w.scores);
+    rc = cuda_code(launch_rowmax(rowmax_args(p, d, xs_q, kc, ws + w.cbf, scores), s));
+    if (rc) return rc;
+    sa.scores = scores;
+    sa.qc = nullptr;
+  }
+  rc = run_select(p, d, sa, ws, w.sigma, w.fire, s);
   if (rc) return rc;
   return launch_attend(attend_args(p, d, q, k, v, idx, cnt, o), s);
 }

@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
 
   for (int e = tid; e < R * DS; e += kSelThreads) {
     const int r = e / DS;
-    qs[e] = (r < rows) ? a.qc[((size_t)hs * a.nb + i0 + r) * DS + (e % DS)] : 0.f;
+    qs[e] = (r < rows && a.qc) ? a.qc[((size_t)hs * a.nb + i0 + r) * DS + (e % DS)] : 0.f;
   }
   __syncthreads();
 
@@ -322,7 +322,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
   // and streams their centroid rows (fp32) from L2 in 16-byte pieces, dotting
   // each piece with the R pooled queries read from shared memory (every lane
   // reads the same address: one broadcast per row).
-  if (a.minmax) {
+  if (a.scores) {
+    // precomputed tile scores (row-max): copy the rows' candidates
+    for (int r = 0; r < rows; ++r) {
+      const float* src = a.scores + ((size_t)hs * a.nb + i0 + r) * a.nb;
+      for (int j = tid; j < i0 + r; j += kSelThreads) sc[r * score_stride + j] = src[j];
+    }
+  } else if (a.minmax) {
     // Upper-bound backbone: s_j = sum_d max(q_d min_jd, q_d max_jd), the two
     // table rows of block j streamed like a centroid row.
     const float* km = a.kc + (size_t)g * a.nb * 2 * DS;
@@ -350,7 +356,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
     }
   }
   const float* kc = a.kc + (size_t)g * a.nb * DS;
-  for (int j = a.minmax ? jend : tid; j < jend; j += kSelThreads) {
+  for (int j = (a.minmax || a.scores) ? jend : tid; j < jend; j += kSelThreads) {
     const float4* crow = reinterpret_cast<const float4*>(kc + (size_t)j * DS);
     float acc[R];
 #pragma unroll

@@ -23,10 +23,12 @@ BF16, FP32 = 0, 1
 TOPK, CUMMASS = 0, 1
 BACKBONE_MEAN, BACKBONE_MINMAX = 0, 1
 GATE_GAP, GATE_PERCENTILE = 1, 2
+TILE_MEAN, TILE_ROWMAX = 0, 1
 FLAG_GATE, FLAG_RESCUE = 1, 2
 
 SYMBOLS = ["sbsa_pool_blocks", "sbsa_pool_minmax", "sbsa_select", "sbsa_select_ws",
-           "sbsa_select_workspace_bytes", "sbsa_attend", "sbsa_prefill",
+           "sbsa_select_workspace_bytes", "sbsa_score_rowmax", "sbsa_score_rowmax_workspace_bytes",
+           "sbsa_select_scores", "sbsa_attend", "sbsa_prefill",
            "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string",
            "sbsa_version", "sbsa_debug_wait_timeout"]
 
@@ -60,6 +62,7 @@ class Params(ctypes.Structure):
         ("backbone", ctypes.c_int),
         ("gate_quantile", ctypes.c_float),
         ("gate_rho", ctypes.c_int),
+        ("tile_score", ctypes.c_int),
     ]
 
     @property
@@ -90,6 +93,10 @@ def _load() -> ctypes.CDLL:
     lib.sbsa_select_ws.argtypes = [P, f32p, f32p, f32p, i32p, i32p, u8p, vp, ctypes.c_size_t, vp]
     lib.sbsa_select_workspace_bytes.argtypes = [P]
     lib.sbsa_select_workspace_bytes.restype = ctypes.c_size_t
+    lib.sbsa_score_rowmax.argtypes = [P, vp, f32p, f32p, vp, ctypes.c_size_t, vp]
+    lib.sbsa_score_rowmax_workspace_bytes.argtypes = [P]
+    lib.sbsa_score_rowmax_workspace_bytes.restype = ctypes.c_size_t
+    lib.sbsa_select_scores.argtypes = [P, f32p, i32p, i32p, u8p, vp, ctypes.c_size_t, vp]
     lib.sbsa_attend.argtypes = [P, vp, vp, vp, i32p, i32p, vp, vp]
     lib.sbsa_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i32p, i32p, u8p, vp]
     lib.sbsa_prefill_workspace_bytes.argtypes = [P]
@@ -144,7 +151,7 @@ def make_params(*, n_q_heads, n_kv_heads, seq_len, head_dim, block_size, dtype="
                 select_mode="topk", top_k=0, mass_threshold=0.0, rescue_tau=None,
                 gate_margin=None, group_shared=False, index_dim=0, max_blocks=None,
                 sm_scale=0.0, score_scale=0.0, backbone="mean", gate_quantile=None,
-                gate_rho=2) -> Params:
+                gate_rho=2, tile_score="mean") -> Params:
     p = Params()
     p.n_q_heads, p.n_kv_heads, p.seq_len = n_q_heads, n_kv_heads, seq_len
     p.head_dim, p.block_size = head_dim, block_size
@@ -163,6 +170,8 @@ def make_params(*, n_q_heads, n_kv_heads, seq_len, head_dim, block_size, dtype="
     p.gate_margin = 0.0 if gate_margin is None else float(gate_margin)
     p.gate_quantile = 0.0 if gate_quantile is None else float(gate_quantile)
     p.gate_rho = int(gate_rho)
+    p.tile_score = ({"mean": TILE_MEAN, "rowmax": TILE_ROWMAX}[tile_score]
+                    if isinstance(tile_score, str) else int(tile_score))
     nb = (seq_len + block_size - 1) // block_size
     if max_blocks is None:
         if p.select_mode == CUMMASS or p.rescue:
@@ -188,7 +197,8 @@ def params_for(w) -> Params:
                        index_dim=w.index_dim, max_blocks=w.max_blocks,
                        backbone=getattr(w, "backbone", "mean"),
                        gate_quantile=getattr(w, "gate_quantile", None),
-                       gate_rho=getattr(w, "gate_rho", 2))
+                       gate_rho=getattr(w, "gate_rho", 2),
+                       tile_score=getattr(w, "tile_score", "mean"))
 
 
 _TORCH_DT = {BF16: torch.bfloat16, FP32: torch.float32}
@@ -241,6 +251,36 @@ def select(p: Params, q_cent: torch.Tensor, k_cent: torch.Tensor,
     _check(lib.sbsa_select_ws(ctypes.byref(p), _ptr(q_cent), _ptr(k_cent),
                               _ptr(k_radius) if p.rescue else None, _ptr(idx), _ptr(cnt),
                               _ptr(flags), _ptr(ws), wsb, _stream(stream)), "sbsa_select_ws")
+    return idx, cnt, flags
+
+
+def score_rowmax(p: Params, q_src: torch.Tensor, k_cent: torch.Tensor, stream=None):
+    """Row-max tile scores [Hs, NB, NB] (entries j < i of row i are defined)."""
+    nb, hs, ds = p.n_blocks, p.n_sel_heads, p.score_dim
+    _need(q_src, "q_src", torch.bfloat16, (p.n_q_heads, p.seq_len, ds))
+    _need(k_cent, "k_cent", torch.float32, (p.n_kv_heads, nb, ds))
+    dev = q_src.device
+    scores = torch.zeros(hs, nb, nb, device=dev, dtype=torch.float32)
+    wsb = int(lib.sbsa_score_rowmax_workspace_bytes(ctypes.byref(p)))
+    ws = torch.empty(max(wsb, 1), device=dev, dtype=torch.uint8)
+    _check(lib.sbsa_score_rowmax(ctypes.byref(p), _ptr(q_src), _ptr(k_cent), _ptr(scores),
+                                 _ptr(ws), wsb, _stream(stream)), "sbsa_score_rowmax")
+    return scores
+
+
+def select_scores(p: Params, scores: torch.Tensor, stream=None):
+    """Block lists from a precomputed tile-score table [Hs, NB, NB]."""
+    nb, hs = p.n_blocks, p.n_sel_heads
+    _need(scores, "scores", torch.float32, (hs, nb, nb))
+    dev = scores.device
+    idx = torch.empty(hs, nb, p.max_blocks, device=dev, dtype=torch.int32)
+    cnt = torch.empty(hs, nb, device=dev, dtype=torch.int32)
+    flags = torch.empty(hs, nb, device=dev, dtype=torch.uint8)
+    wsb = int(lib.sbsa_select_workspace_bytes(ctypes.byref(p)))
+    ws = torch.empty(wsb, device=dev, dtype=torch.uint8) if wsb else None
+    _check(lib.sbsa_select_scores(ctypes.byref(p), _ptr(scores), _ptr(idx), _ptr(cnt),
+                                  _ptr(flags), _ptr(ws), wsb, _stream(stream)),
+           "sbsa_select_scores")
     return idx, cnt, flags
 
 
@@ -339,6 +379,11 @@ class Staged:
         self.idx = torch.empty(hs, nb, p.max_blocks, device=device, dtype=torch.int32)
         self.cnt = torch.empty(hs, nb, device=device, dtype=torch.int32)
         self.flags = torch.empty(hs, nb, device=device, dtype=torch.uint8)
+        self.rowmax = p.tile_score == TILE_ROWMAX
+        self.scores = torch.empty(hs, nb, nb, **f32) if self.rowmax else None
+        self.rm_bytes = int(lib.sbsa_score_rowmax_workspace_bytes(ctypes.byref(p)))
+        self.rm_ws = (torch.empty(self.rm_bytes, device=device, dtype=torch.uint8)
+                      if self.rowmax else None)
         self.ws_bytes = int(lib.sbsa_select_workspace_bytes(ctypes.byref(p)))
         self.ws = (torch.empty(self.ws_bytes, device=device, dtype=torch.uint8)
                    if self.ws_bytes else None)
@@ -354,10 +399,20 @@ class Staged:
         else:
             _check(lib.sbsa_pool_blocks(self._p, _ptr(k_src), p.n_kv_heads, ds, 1, _ptr(self.kc),
                                         _ptr(self.kr), s), "sbsa_pool_blocks")
+        if self.rowmax:
+            # the tile scores read the query rows themselves
+            _check(lib.sbsa_score_rowmax(self._p, _ptr(q_src), _ptr(self.kc), _ptr(self.scores),
+                                         _ptr(self.rm_ws), self.rm_bytes, s), "sbsa_score_rowmax")
+            return
         _check(lib.sbsa_pool_blocks(self._p, _ptr(q_src), p.n_q_heads, ds, grp, _ptr(self.qc),
                                     None, s), "sbsa_pool_blocks")
 
     def select(self, stream=None):
+        if self.rowmax:
+            _check(lib.sbsa_select_scores(self._p, _ptr(self.scores), _ptr(self.idx),
+                                          _ptr(self.cnt), _ptr(self.flags), _ptr(self.ws),
+                                          self.ws_bytes, _stream(stream)), "sbsa_select_scores")
+            return
         _check(lib.sbsa_select_ws(self._p, _ptr(self.qc), _ptr(self.kc), _ptr(self.kr),
                                   _ptr(self.idx), _ptr(self.cnt), _ptr(self.flags),
                                   _ptr(self.ws), self.ws_bytes, _stream(stream)),

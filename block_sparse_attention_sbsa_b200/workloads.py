@@ -28,6 +28,9 @@ Five workload families, one per configuration of the benchmark suite:
 * ``quest32k`` 32/8 heads, d=128, N=32768, B=128, bf16, top-16 per query head
               scored by the K-min/K-max upper bound; the RBS recipe's clustered
               keys with outliers, whose blocks the bound is designed to catch.
+* ``rowmax32k`` the GQA-32k recipe (32/8 heads, top-16 per query head) with
+              the page's tile score: the largest q_t . c_j over the tile's
+              query rows (a tensor-core contraction) instead of the pooled query.
 * ``sigma64k`` the gate recipe at 64k (32/8 heads, B=64, top-8) with the
               page's own gate instead of the gap test: tiles whose head-averaged
               normalised cut margin is in the lowest 30% take the top 16.
@@ -66,6 +69,7 @@ class Workload:
     backbone: str = "mean"          # "mean" (centroids) | "minmax" (K-min/K-max bound)
     gate_quantile: Optional[float] = None  # the page's percentile gate: q ...
     gate_rho: int = 2                      # ... and the expansion factor rho
+    tile_score: str = "mean"               # "mean" (pooled query) | "rowmax" (max over rows)
 
     @property
     def n_blocks(self) -> int:
@@ -115,6 +119,8 @@ CONFIGS = {
                          top_k=16, seed=1006, backbone="minmax"),
     "sigma64k": Workload("sigma64k", "gate", 32, 8, 65536, 128, 64, "bf16", "topk",
                          top_k=8, seed=1004, gate_quantile=0.3, gate_rho=2),
+    "rowmax32k": Workload("rowmax32k", "gqa", 32, 8, 32768, 128, 128, "bf16", "topk",
+                          top_k=16, seed=1002, tile_score="rowmax"),
 }
 
 # Reduced shapes of the same recipes, small enough for the CPU oracle to
@@ -139,6 +145,11 @@ SMALL = {
                                                    gate_margin=0.05),
     "sigma_small": CONFIGS["sigma64k"].scaled(name="sigma_small", n_q_heads=4, n_kv_heads=2,
                                               seq_len=8192),
+    "rowmax_small": CONFIGS["rowmax32k"].scaled(name="rowmax_small", n_q_heads=4,
+                                                n_kv_heads=2, seq_len=4096 + 77, top_k=8),
+    "rowmax_msa_small": CONFIGS["msa512k"].scaled(name="rowmax_msa_small", n_q_heads=8,
+                                                  n_kv_heads=2, seq_len=8192 + 100, top_k=8,
+                                                  tile_score="rowmax"),
     "sigma_quest_small": CONFIGS["quest32k"].scaled(name="sigma_quest_small", n_q_heads=4,
                                                     n_kv_heads=2, seq_len=8192 + 50, top_k=8,
                                                     gate_quantile=0.5, gate_rho=3),

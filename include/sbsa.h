@@ -97,7 +97,15 @@ typedef struct sbsa_params {
                            excludes the rescue branch (which needs radii)    */
   float gate_quantile;  /* SBSA_GATE_PERCENTILE: q in [0, 1]                  */
   int gate_rho;         /* SBSA_GATE_PERCENTILE: fired tiles take rho*k, rho >= 1 */
+  int tile_score;       /* SBSA_TILE_MEAN | SBSA_TILE_ROWMAX; ROWMAX needs the
+                           mean backbone, bf16 inputs and no rescue branch   */
 } sbsa_params;
+
+/* ---- query side of a tile score ([UGS] Metodologia step 2) ---- */
+#define SBSA_TILE_MEAN 0   /* the pooled (mean) query of the tile: one dot per block     */
+#define SBSA_TILE_ROWMAX 1 /* the page's tile score: the largest q_t . c_j over the
+                              tile's query rows (and, per GQA group, the group's heads),
+                              a tensor-core contraction; centroids enter as bf16 */
 
 /* ---- gates ([UGS] Metodologia steps 3-5) ---- */
 #define SBSA_GATE_GAP 1        /* per row: gap at the cut below margin * std -> 2k   */
@@ -161,6 +169,31 @@ int sbsa_select(const sbsa_params* p, const float* q_cent, const float* k_cent,
  * score_scale; everything else is unchanged.  With p->gate ==
  * SBSA_GATE_PERCENTILE sbsa_select returns SBSA_ERR_WORKSPACE: use
  * sbsa_select_ws. */
+
+/*
+ * sbsa_score_rowmax -- the page's tile scores (SBSA_TILE_ROWMAX).
+ *   q_src    device [Hq, N, ds] bf16: Q, or Q_idx when p->index_dim is set.
+ *   k_cent   device fp32 [Hkv, NB, ds] key centroids (sbsa_pool_blocks).
+ *   scores   device fp32 [Hs, NB, NB] out: scores[hs, i, j] for j < i is
+ *            max_t (q_t . bf16(c_j)) * score_scale over the query rows t of
+ *            block i (rows t < N) of head hs, or of every head of group hs
+ *            when p->group_shared; entries j >= i are not written.
+ *   workspace device, 256-byte aligned, >= sbsa_score_rowmax_workspace_bytes(p)
+ *            (the bf16 copy of the centroids).
+ * Errors as sbsa_select, plus SBSA_ERR_UNSUPPORTED when p->tile_score is not
+ * SBSA_TILE_ROWMAX.
+ */
+size_t sbsa_score_rowmax_workspace_bytes(const sbsa_params* p);
+int sbsa_score_rowmax(const sbsa_params* p, const void* q_src, const float* k_cent,
+                      float* scores, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * sbsa_select_scores -- sbsa_select_ws on precomputed tile scores
+ * [Hs, NB, NB] (sbsa_score_rowmax) instead of pooled tables; every rule
+ * (top-k, the gates, cumulative mass, the diagonal) applies unchanged.
+ */
+int sbsa_select_scores(const sbsa_params* p, const float* scores, int32_t* idx, int32_t* cnt,
+                       uint8_t* flags, void* workspace, size_t ws_bytes, void* stream);
 
 /* Device workspace sbsa_select_ws needs (0 when no gate needs one; also 0
  * when p is invalid). */

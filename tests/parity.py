@@ -126,12 +126,13 @@ def row_matches(gpu_ids, s, ub, i, w, budgets_i=None):
 
 
 def compare_lists(gpu_idx, gpu_cnt, oracle_idx, oracle_cnt, rows, qbar, c, r, w, kv_of_sel,
-                  minmax=None, budgets=None):
+                  minmax=None, budgets=None, score_fn=None):
     """Returns (exact, tie) counts over ``rows``; raises AssertionError on a
     difference the tie band does not explain.  ``minmax`` = (kmin, kmax)
     selects the upper-bound backbone's scores instead of the centroids';
     ``budgets`` (tile -> allowed top-k budgets) carries the percentile gate's
-    decisions."""
+    decisions; ``score_fn(hs, i)`` gives the oracle's scores of a row
+    directly (row-max tile scores)."""
     exact = tie = 0
     scale = 1.0 / math.sqrt(w.score_dim)
     for (hs, i) in rows:
@@ -141,7 +142,9 @@ def compare_lists(gpu_idx, gpu_cnt, oracle_idx, oracle_cnt, rows, qbar, c, r, w,
             exact += 1
             continue
         g = kv_of_sel(hs)
-        if minmax is None:
+        if score_fn is not None:
+            s = score_fn(hs, i)
+        elif minmax is None:
             s = O.block_scores(qbar[hs, i], c[g], i, scale)
         else:
             s = O.block_bounds_minmax(qbar[hs, i], minmax[0][g], minmax[1][g], i, scale)

@@ -56,7 +56,7 @@ int main(void) {
   F(n_q_heads) F(n_kv_heads) F(seq_len) F(head_dim) F(block_size) F(dtype) F(select_mode)
   F(group_shared) F(index_dim) F(top_k) F(mass_threshold) F(rescue) F(rescue_tau) F(gate)
   F(gate_margin) F(max_blocks) F(sm_scale) F(score_scale) F(backbone) F(gate_quantile)
-  F(gate_rho)
+  F(gate_rho) F(tile_score)
   return 0;
 }
 '''
@@ -116,6 +116,10 @@ def _attend(sb, p):
     (dict(gate_quantile=0.3, gate_rho=0), 1),
     (dict(gate_quantile=0.3, gate_rho=3, max_blocks=7), 1),   # needs min(rho*k, NB-1)+1 = 8
     (dict(select_mode="cummass", mass_threshold=0.9, gate_quantile=0.3), 1),
+    (dict(tile_score=2), 1),                     # no such tile score
+    (dict(tile_score="rowmax", backbone="minmax"), 1),
+    (dict(tile_score="rowmax", dtype="fp32"), 1),
+    (dict(tile_score="rowmax", select_mode="cummass", mass_threshold=0.9, rescue_tau=1.0), 1),
     (dict(select_mode="cummass", mass_threshold=0.9, rescue_tau=5.0, backbone="minmax"), 1),
 ])
 def test_invalid_parameters_are_rejected_before_launch(sb, mutate, code):
@@ -183,6 +187,22 @@ def test_percentile_gate_needs_a_workspace(sb):
     # the prefill workspace grows by the same scratch
     plain = sb.workspace_bytes(_valid(sb, seq_len=4096, max_blocks=p.max_blocks))
     assert sb.workspace_bytes(p) == plain + need
+
+
+def test_rowmax_workspace_and_checks(sb):
+    p = _valid(sb, tile_score="rowmax", seq_len=4096)
+    nb = p.n_blocks
+    need = sb.lib.sbsa_score_rowmax_workspace_bytes(ctypes.byref(p))
+    assert need == (2 * nb * 128 * 2 + 255) // 256 * 256
+    assert sb.lib.sbsa_score_rowmax_workspace_bytes(ctypes.byref(_valid(sb))) == 0
+    f = sb.lib.sbsa_score_rowmax
+    assert f(ctypes.byref(_valid(sb)), FAKE, FAKE, FAKE, FAKE, need, None) == 2  # not rowmax
+    assert f(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, need - 1, None) == 3
+    assert f(ctypes.byref(p), None, FAKE, FAKE, FAKE, need, None) == 1
+    # the prefill workspace holds the bf16 centroids and the score table too
+    plain = sb.workspace_bytes(_valid(sb, seq_len=4096))
+    scores = (4 * nb * nb * 4 + 255) // 256 * 256
+    assert sb.workspace_bytes(p) >= plain + need + scores - 256
 
 
 def test_fp32_attention_is_limited_to_d64_b64(sb):

@@ -15,7 +15,8 @@ from block_sparse_attention_sbsa_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 SMALL_NAMES = ["tiny", "gqa_small", "rbs_small", "gate_small", "msa_small", "quest_small",
-               "quest_gate_small", "sigma_small", "sigma_quest_small"]
+               "quest_gate_small", "sigma_small", "sigma_quest_small", "rowmax_small",
+               "rowmax_msa_small"]
 
 
 @pytest.fixture(scope="module")
@@ -43,7 +44,7 @@ def _oracle_prefill(w, data, **kw):
                      top_k_=w.top_k, mass=w.mass_threshold, margin=w.gate_margin,
                      tau=w.rescue_tau, group_shared=w.group_shared, q_idx=data["q_idx"],
                      k_idx=data["k_idx"], max_blocks=w.max_blocks, backbone=w.backbone,
-                     sigma_gate=_sigma_gate(w), **kw)
+                     sigma_gate=_sigma_gate(w), tile_score=w.tile_score, **kw)
 
 
 @functools.lru_cache(maxsize=None)
@@ -51,6 +52,27 @@ def small_case(name):
     w = W.SMALL[name]
     data = W.generate(w, "cpu")
     return w, data, _oracle_prefill(w, data)
+
+
+def _rowmax_fn(w, qs_cpu, c):
+    """Oracle row-max tile scores of row (hs, i), or None for pooled queries."""
+    if w.tile_score != "rowmax":
+        return None
+    scale = 1.0 / math.sqrt(w.score_dim)
+    b = w.block_size
+
+    def fn(hs, i):
+        heads = range(hs * w.group, (hs + 1) * w.group) if w.group_shared else [hs]
+        rows = np.concatenate([np.asarray(qs_cpu[h, i * b:min(w.seq_len, (i + 1) * b)].double())
+                               for h in heads])
+        g = hs if w.group_shared else hs // w.group
+        return O.block_scores_rowmax(rows, c[g], i, scale)
+    return fn
+
+
+def _small_rowmax_fn(w, data, ref):
+    qs = data["q_idx"] if w.index_dim else data["q"]
+    return _rowmax_fn(w, qs, ref["c"])
 
 
 def _dev(data):
@@ -98,11 +120,20 @@ def test_select_on_oracle_tables(sb, name):
     else:
         kc = torch.tensor(ref["c"], dtype=torch.float32, device="cuda")
     kr = torch.tensor(ref["r"], dtype=torch.float32, device="cuda")
-    idx, cnt, flags = sb.select(p, qc, kc, kr if w.rescue_tau is not None else None)
+    if w.tile_score == "rowmax":
+        # the oracle's tile-score table in, lists out
+        fn = _small_rowmax_fn(w, data, ref)
+        table = np.zeros((w.n_sel_heads, w.n_blocks, w.n_blocks), dtype=np.float32)
+        for hs in range(w.n_sel_heads):
+            for i in range(1, w.n_blocks):
+                table[hs, i, :i] = fn(hs, i)
+        idx, cnt, flags = sb.select_scores(p, torch.tensor(table, device="cuda"))
+    else:
+        idx, cnt, flags = sb.select(p, qc, kc, kr if w.rescue_tau is not None else None)
     idx, cnt, flags = idx.cpu().numpy(), cnt.cpu().numpy(), flags.cpu().numpy()
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
                                   ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"],
-                                  budgets=_budgets(w, ref))
+                                  budgets=_budgets(w, ref), score_fn=_small_rowmax_fn(w, data, ref))
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # padding and flags
     for hs in range(w.n_sel_heads):
@@ -139,7 +170,7 @@ def test_prefill_end_to_end(sb, name):
     idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
                                   ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"],
-                                  budgets=_budgets(w, ref))
+                                  budgets=_budgets(w, ref), score_fn=_small_rowmax_fn(w, data, ref))
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # outputs on query rows whose lists match the oracle exactly
     o = o.float().cpu().numpy()
@@ -154,6 +185,27 @@ def test_prefill_end_to_end(sb, name):
     assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
 
 
+@pytest.mark.parametrize("name", ["rowmax_small", "rowmax_msa_small"])
+def test_rowmax_tile_scores_match_oracle(sb, name):
+    """The tensor-core row-max scores against the oracle's (bf16 centroids,
+    exact products, float64 sums) for every (selection head, tile, j < i)."""
+    w, data, ref = small_case(name)
+    p = sb.params_for(w)
+    d = _dev(data)
+    qs = d["q_idx"] if w.index_dim else d["q"]
+    kc = torch.tensor(ref["c"], dtype=torch.float32, device="cuda")
+    got = sb.score_rowmax(p, qs, kc).cpu().numpy()
+    assert sb.get_status() == sb.OK
+    fn = _small_rowmax_fn(w, data, ref)
+    worst = 0.0
+    for hs in range(w.n_sel_heads):
+        for i in range(1, w.n_blocks):
+            want = fn(hs, i).astype(np.float64)
+            err = np.abs(got[hs, i, :i] - want) / np.maximum(1.0, np.abs(want))
+            worst = max(worst, float(err.max()))
+    assert worst <= PT.BAND, worst
+
+
 def test_gate_fires_on_the_planted_rows(sb):
     w, data, ref = small_case("gate_small")
     p = sb.params_for(w)
@@ -165,7 +217,7 @@ def test_gate_fires_on_the_planted_rows(sb):
 
 # ------------------------------------------------------------- full sizes
 
-FULL = ["gqa32k", "rbs128k", "gate64k", "msa512k", "quest32k", "sigma64k"]
+FULL = ["gqa32k", "rbs128k", "gate64k", "msa512k", "quest32k", "sigma64k", "rowmax32k"]
 
 
 def _sample_blocks(w, meta, count):
@@ -197,6 +249,7 @@ def test_full_size_sampled(sb, name):
     if r is None:
         r = np.zeros(c.shape[:2])
     mmx = O.pool_keys_minmax(ks, w.block_size) if w.backbone == "minmax" else None
+    rfn = _rowmax_fn(w, (data["q_idx"] if w.index_dim else data["q"]).cpu(), c)
     nb = w.n_blocks
     qrows = torch.cat([qs[:, i * w.block_size:(i + 1) * w.block_size] for i in blocks], dim=1).cpu()
     # pooled queries of the sampled blocks only (of every block when the
@@ -215,7 +268,7 @@ def test_full_size_sampled(sb, name):
                                mass=w.mass_threshold, margin=w.gate_margin, tau=w.rescue_tau,
                                scale=1.0 / math.sqrt(w.score_dim), kv_of_sel=_kv_of_sel(w),
                                max_blocks=w.max_blocks, rows=sel_rows, minmax=mmx,
-                               sigma_gate=_sigma_gate(w), info=info)
+                               sigma_gate=_sigma_gate(w), info=info, row_scores=rfn)
     gidx = call.idx[:, blocks].cpu().numpy()
     gcnt = call.cnt[:, blocks].cpu().numpy()
     gi_full = np.full((w.n_sel_heads, nb, w.max_blocks), -1, dtype=np.int32)
@@ -223,7 +276,8 @@ def test_full_size_sampled(sb, name):
     gi_full[:, blocks] = gidx
     gc_full[:, blocks] = gcnt
     exact, tie = PT.compare_lists(gi_full, gc_full, idx, cnt, sel_rows, qbar, c, r, w,
-                                  _kv_of_sel(w), minmax=mmx, budgets=_budgets(w, info))
+                                  _kv_of_sel(w), minmax=mmx, budgets=_budgets(w, info),
+                                  score_fn=rfn)
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # outputs of the sampled blocks whose lists match (all query heads; two
     # per group for the 64-head workload); keys/values converted once per
