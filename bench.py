@@ -193,20 +193,43 @@ def oracle_sample(w, data_cpu, blocks):
     c, r = O.pool_keys(ks, w.block_size, with_radius=w.rescue_tau is not None)
     if r is None:
         r = np.zeros(c.shape[:2])
-    t_pool = time.perf_counter() - t0
-    t1 = time.perf_counter()
+    minmax = O.pool_keys_minmax(ks, w.block_size) if w.backbone == "minmax" else None
     nb, b = w.n_blocks, w.block_size
     grp = w.group if w.group_shared else 1
     qbar = np.zeros((w.n_sel_heads, nb, w.score_dim))
+    sigma_gate, fired = None, None
+    kv_of = (lambda hs: hs) if w.group_shared else (lambda hs: hs // w.group)
+    if w.gate_quantile is not None:
+        # the gate's global part (every tile's margin and the tile decisions)
+        # is per prefill, not per block
+        qbar = O.pool_queries(data_cpu["q_all"], b, group=grp)
+        sigma_gate = (w.gate_quantile, w.gate_rho)
+        info = {}
+        O.select(qbar, c, r, block_count=nb, mode=w.select_mode, top_k_=w.top_k,
+                 scale=1.0 / math.sqrt(w.score_dim), kv_of_sel=kv_of, max_blocks=w.max_blocks,
+                 rows=[], minmax=minmax, sigma_gate=sigma_gate, info=info)
+        fired = info["fired"]
+    t_pool = time.perf_counter() - t0
+    t1 = time.perf_counter()
     qsrc = data_cpu["q_rows_idx"] if w.index_dim else data_cpu["q_rows"]
     for bi, i in enumerate(blocks):
         qbar[:, i] = O.pool_queries(qsrc[:, bi * b:(bi + 1) * b], b, group=grp)[:, 0]
-    kv_of = (lambda hs: hs) if w.group_shared else (lambda hs: hs // w.group)
     rows = [(hs, i) for hs in range(w.n_sel_heads) for i in blocks]
+    row_scores = None
+    if w.tile_score == "rowmax":
+        where = {i: bi for bi, i in enumerate(blocks)}
+
+        def row_scores(hs, i):
+            heads = range(hs * grp, (hs + 1) * grp) if w.group_shared else [hs]
+            bi = where[i]
+            tile = np.concatenate([np.asarray(qsrc[h, bi * b:(bi + 1) * b].double())
+                                   for h in heads])
+            return O.block_scores_rowmax(tile, c[kv_of(hs)], i, 1.0 / math.sqrt(w.score_dim))
     idx, cnt, _ = O.select(qbar, c, r, block_count=nb, mode=w.select_mode, top_k_=w.top_k,
                            mass=w.mass_threshold, margin=w.gate_margin, tau=w.rescue_tau,
                            scale=1.0 / math.sqrt(w.score_dim), kv_of_sel=kv_of,
-                           max_blocks=w.max_blocks, rows=rows)
+                           max_blocks=w.max_blocks, rows=rows, minmax=minmax,
+                           sigma_gate=sigma_gate, row_scores=row_scores, fired=fired)
     scale = 1.0 / math.sqrt(w.head_dim)
     for bi, i in enumerate(blocks):
         for h in range(w.n_q_heads):
@@ -227,6 +250,9 @@ def cpu_copy_for_oracle(w, data, blocks):
     if data["q_idx"] is not None:
         out["q_rows_idx"] = torch.cat([data["q_idx"][:, i * b:(i + 1) * b] for i in blocks],
                                       dim=1).cpu()
+    if w.gate_quantile is not None:
+        # the percentile gate ranks every tile: the oracle needs every query block
+        out["q_all"] = (data["q_idx"] if data["q_idx"] is not None else data["q"]).cpu()
     return out
 
 
@@ -298,15 +324,27 @@ def run_reference(args):
     return 0
 
 
-def workload_config(w):
+def workload_config(w, world: int = 1, heads: bool = False):
+    if w.select_mode == "cummass":
+        sel = f"cumulative mass {w.mass_threshold} + rescue tau {w.rescue_tau}"
+    else:
+        sel = f"top-{w.top_k}"
+        if w.gate_margin is not None:
+            sel += f" gated x2 margin {w.gate_margin}"
+        if w.gate_quantile is not None:
+            sel += f" percentile gate q {w.gate_quantile} rho {w.gate_rho}"
+        if w.group_shared:
+            sel += " per GQA group"
+    if w.backbone != "mean":
+        sel += ", K-min/K-max upper-bound scores"
+    if w.tile_score != "mean":
+        sel += ", row-max tile scores"
     return {"workload": w.name, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
             "seq_len": w.seq_len, "head_dim": w.head_dim, "block_size": w.block_size,
-            "select": (f"cumulative mass {w.mass_threshold} + rescue tau {w.rescue_tau}"
-                       if w.select_mode == "cummass" else
-                       f"top-{w.top_k}" + (f" gated x2 margin {w.gate_margin}" if w.gate_margin
-                                           else "") + (" per GQA group" if w.group_shared else "")),
-            "global_batch": 1, "seq": w.seq_len,
-            "l2": "inputs larger than L2 (Q, K, V each exceed 126 MB); no flush between steps"}
+            "select": sel, "global_batch": 1, "seq": w.seq_len,
+            "l2": "inputs larger than L2 (Q, K, V each exceed 126 MB); no flush between steps",
+            "parallelism": (f"kv heads split over {world} GPUs" if heads else
+                            f"{world} independent sequence(s), one per GPU")}
 
 
 # ------------------------------------------------------- rank bookkeeping
@@ -506,9 +544,7 @@ def main():
         "scaling": "strong" if heads else "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "fp32",
         "data": "synthetic (seeded generator, RBS-style clustered keys with outliers)",
-        "config": dict(workload_config(w_full),
-                       parallelism=(f"kv heads split over {world} GPUs" if heads else
-                                    f"{world} independent sequence(s), one per GPU")),
+        "config": workload_config(w_full, world, heads),
         "attended_tflops": att_tflops,
         "roofline": {
             "bound": "tensor", "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",

@@ -300,7 +300,7 @@ def select_row(s, i: int, *, mode: str, top_k_: int = 0, mass: float = 0.0,
 def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
            mass: float = 0.0, margin=None, tau=None, scale: float,
            kv_of_sel=None, max_blocks: int, rows=None, minmax=None, sigma_gate=None,
-           info=None, row_scores=None):
+           info=None, row_scores=None, fired=None):
     """Lists for every selection head hs and query block i (or the (hs, i)
     pairs in ``rows``).  ``qbar`` is [Hs, NB, d_s] and ``c``/``r`` are the key
     tables [Hkv, NB, ...]; ``kv_of_sel(hs)`` gives the kv head whose key table
@@ -321,8 +321,9 @@ def select(qbar, c, r, *, block_count: int, mode: str, top_k_: int = 0,
             return block_scores(qbar[h, i], c[g], i, scale)
         return block_bounds_minmax(qbar[h, i], minmax[0][g], minmax[1][g], i, scale)
 
-    fired = set()
-    if sigma_gate is not None:
+    given_fired = fired is not None
+    fired = set(fired) if given_fired else set()  # the gate's tiles, when decided earlier
+    if sigma_gate is not None and not given_fired:
         if mode != "topk" or margin is not None:
             raise ValueError("the percentile gate applies to plain top-k")
         q, rho = sigma_gate
