@@ -91,6 +91,20 @@ def attend_kernel_name(w) -> str:
     return f"attend_kernel (one CTA per query block, tcgen05, {shape})"
 
 
+def launches_per_step(w) -> int:
+    """Kernels one staged prefill step launches (the calls of sbsa.Staged):
+    key pooling; query pooling, or the bf16 conversion and row-max scores;
+    with the mean backbone and mean tile scores the tf32 split and the
+    tensor-core centroid scores; the selection (three launches under the
+    percentile gate); the attention."""
+    rowmax = w.tile_score == "rowmax"
+    n = 1 + (2 if rowmax else 1)
+    if w.backbone == "mean" and not rowmax and w.n_blocks >= 2:
+        n += 2
+    n += 3 if w.gate_quantile is not None else 1
+    return n + 1
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -568,7 +582,7 @@ def main():
                     "far below the HBM peak: attention is not bound by DRAM",
         },
         "attended_pairs": pairs,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": launches_per_step(w) * args.steps,
         "clocks": clk,
         "e2e": {"value": weak_throughput(w.seq_len, world, args.e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

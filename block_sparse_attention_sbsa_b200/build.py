@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsbsa.so")
-SOURCES = ["pool.cu", "select.cu", "score_rowmax.cu", "attend.cu", "attend_persist.cu",
+SOURCES = ["pool.cu", "select.cu", "score_rowmax.cu", "score_centroid.cu", "attend.cu",
+           "attend_persist.cu",
            "attend_pair.cu",
            "sbsa_api.cu",
            "sbsa_noalloc.cu"]

@@ -44,7 +44,7 @@ struct SelectArgs {
   int rho;
   double* sigma;        // [Hs, NB] cut margins (NaN: no cut), written by pass 1
   const uint8_t* fire;  // [NB] 1 for fired tiles, read by pass 2
-  const float* scores;  // [Hs, NB, NB] precomputed tile scores (row-max), or nullptr
+  const float* scores;  // [Hs, NB, NB] precomputed scores (centroid or row-max), or nullptr
   int top_k;
   float mass;
   int gate;
@@ -75,6 +75,23 @@ struct RowmaxArgs {
   int* status;
 };
 cudaError_t launch_rowmax(const RowmaxArgs& a, cudaStream_t stream);
+
+// Centroid block scores on the tensor cores: qc and kc are split into tf32
+// hi / lo parts (scratch), then scores[hs, i, j] = qc[hs, i] . kc[hs / kv_div, j]
+// * scale for j < i, to fp32 accuracy from three tf32 products.
+struct CentroidScoreArgs {
+  const float* qc;     // [Hs, NB, ds] pooled queries
+  const float* kc;     // [Hkv, NB, ds] centroids
+  float* q_hi;         // [Hs, NB, ds] scratch
+  float* q_lo;         // [Hs, NB, ds] scratch
+  float* c_hi;         // [Hkv, NB, ds] scratch
+  float* c_lo;         // [Hkv, NB, ds] scratch
+  float* scores;       // [Hs, NB, NB]
+  int hs, hkv, kv_div, nb, ds;
+  float scale;
+  int* status;
+};
+cudaError_t launch_centroid_scores(const CentroidScoreArgs& a, cudaStream_t stream);
 
 struct AttendArgs {
   const void* q;

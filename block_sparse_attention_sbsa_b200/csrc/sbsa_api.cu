@@ -108,20 +108,44 @@ int attend_supported(const sbsa_params* p) {
   return SBSA_OK;
 }
 
-struct WsLayout {
-  size_t qc, kc, kr, idx, cnt, flags, sigma, fire, cbf, scores, total;
+// Centroid scores run as a tensor-core product (with the mean backbone and
+// mean tile scores) wherever a workspace holds their scratch.
+bool centroid_tc(const sbsa_params* p) {
+  return p->backbone == SBSA_BACKBONE_MEAN && p->tile_score == SBSA_TILE_MEAN;
+}
+
+// Scratch of a precomputed score table, placed from offset `off`: for the
+// row-max tile scores the bf16 centroids, for the tensor-core centroid
+// scores the tf32 hi / lo parts of the pooled queries and the centroids;
+// then the table [Hs, NB, NB].
+struct ScoreScratch {
+  size_t cbf, q_hi, q_lo, c_hi, c_lo, scores;
 };
 
-// Scratch of the row-max tile scores: the bf16 centroids and the score table.
-size_t rowmax_scratch(const sbsa_params* p, const Derived& d, size_t off, size_t* cbf,
-                      size_t* scores) {
-  const bool on = p->tile_score == SBSA_TILE_ROWMAX;
-  *cbf = off;
-  if (on) off = round_up(off + (size_t)p->n_kv_heads * d.nb * d.ds * 2, 256);
-  *scores = off;
-  if (on) off = round_up(off + (size_t)d.hs * d.nb * d.nb * 4, 256);
+size_t score_scratch(const sbsa_params* p, const Derived& d, size_t off, ScoreScratch* o) {
+  const bool rowmax = p->tile_score == SBSA_TILE_ROWMAX;
+  const bool tc = centroid_tc(p);
+  const size_t q_bytes = (size_t)d.hs * d.nb * d.ds * 4;
+  const size_t c_bytes = (size_t)p->n_kv_heads * d.nb * d.ds * 4;
+  o->cbf = off;
+  if (rowmax) off = round_up(off + c_bytes / 2, 256);
+  o->q_hi = off;
+  if (tc) off = round_up(off + q_bytes, 256);
+  o->q_lo = off;
+  if (tc) off = round_up(off + q_bytes, 256);
+  o->c_hi = off;
+  if (tc) off = round_up(off + c_bytes, 256);
+  o->c_lo = off;
+  if (tc) off = round_up(off + c_bytes, 256);
+  o->scores = off;
+  if (rowmax || tc) off = round_up(off + (size_t)d.hs * d.nb * d.nb * 4, 256);
   return off;
 }
+
+struct WsLayout {
+  size_t qc, kc, kr, idx, cnt, flags, sigma, fire, total;
+  ScoreScratch sc;
+};
 
 // Scratch of the percentile gate: per-row margins (double) and per-tile
 // decisions, placed from offset `off`.
@@ -151,7 +175,7 @@ WsLayout layout(const sbsa_params* p, const Derived& d, bool lists) {
   w.flags = off;
   off = round_up(off + (lists ? (size_t)d.hs * d.nb : 0), 256);
   off = gate_scratch(p, d, off, &w.sigma, &w.fire);
-  off = rowmax_scratch(p, d, off, &w.cbf, &w.scores);
+  off = score_scratch(p, d, off, &w.sc);
   w.total = off;
   return w;
 }
@@ -182,6 +206,27 @@ SelectArgs select_args(const sbsa_params* p, const Derived& d, const float* qc, 
   a.rescue = p->rescue ? 1 : 0;
   a.tau = p->rescue_tau;
   a.score_scale = d.score_scale;
+  a.status = device_status_ptr();
+  return a;
+}
+
+CentroidScoreArgs centroid_args(const sbsa_params* p, const Derived& d, const float* qc,
+                                const float* kc, unsigned char* scratch, const ScoreScratch& o,
+                                float* scores) {
+  CentroidScoreArgs a{};
+  a.qc = qc;
+  a.kc = kc;
+  a.q_hi = reinterpret_cast<float*>(scratch + o.q_hi);
+  a.q_lo = reinterpret_cast<float*>(scratch + o.q_lo);
+  a.c_hi = reinterpret_cast<float*>(scratch + o.c_hi);
+  a.c_lo = reinterpret_cast<float*>(scratch + o.c_lo);
+  a.scores = scores;
+  a.hs = d.hs;
+  a.hkv = p->n_kv_heads;
+  a.kv_div = p->group_shared ? 1 : d.group;
+  a.nb = d.nb;
+  a.ds = d.ds;
+  a.scale = d.score_scale;
   a.status = device_status_ptr();
   return a;
 }
@@ -233,7 +278,7 @@ using namespace sbsa;
 
 extern "C" {
 
-int sbsa_version(void) { return 103; }
+int sbsa_version(void) { return 104; }
 
 const char* sbsa_status_string(int code) {
   switch (code) {
@@ -296,7 +341,35 @@ size_t sbsa_select_workspace_bytes(const sbsa_params* p) {
   Derived d;
   if (validate(p, &d) != SBSA_OK) return 0;
   size_t sigma, fire;
-  return gate_scratch(p, d, 0, &sigma, &fire);
+  ScoreScratch sc;
+  const size_t off = gate_scratch(p, d, 0, &sigma, &fire);
+  return centroid_tc(p) ? score_scratch(p, d, off, &sc) : off;
+}
+
+size_t sbsa_score_centroids_workspace_bytes(const sbsa_params* p) {
+  Derived d;
+  if (validate(p, &d) != SBSA_OK || !centroid_tc(p)) return 0;
+  ScoreScratch sc;
+  score_scratch(p, d, 0, &sc);
+  return sc.scores;  // the split parts; the table is the caller's
+}
+
+int sbsa_score_centroids(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                         float* scores, void* workspace, size_t ws_bytes, void* stream) {
+  Derived d;
+  int rc = validate(p, &d);
+  if (rc) return rc;
+  if (!centroid_tc(p)) return SBSA_ERR_UNSUPPORTED;
+  if (!q_cent || !k_cent || !scores) return SBSA_ERR_INVALID_ARG;
+  if (!aligned16(q_cent) || !aligned16(k_cent) || !aligned16(scores)) return SBSA_ERR_INVALID_ARG;
+  const size_t need = sbsa_score_centroids_workspace_bytes(p);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < need)
+    return SBSA_ERR_WORKSPACE;
+  ScoreScratch sc;
+  score_scratch(p, d, 0, &sc);
+  return cuda_code(launch_centroid_scores(
+      centroid_args(p, d, q_cent, k_cent, static_cast<unsigned char*>(workspace), sc, scores),
+      static_cast<cudaStream_t>(stream)));
 }
 
 size_t sbsa_score_rowmax_workspace_bytes(const sbsa_params* p) {
@@ -367,15 +440,25 @@ int sbsa_select_ws(const sbsa_params* p, const float* q_cent, const float* k_cen
   if (!q_cent || !k_cent || !idx || !cnt) return SBSA_ERR_INVALID_ARG;
   if (p->rescue && !k_radius) return SBSA_ERR_INVALID_ARG;
   if (!aligned16(q_cent) || !aligned16(k_cent)) return SBSA_ERR_INVALID_ARG;
+  // workspace: the percentile gate's scratch, then the score table's
   size_t sigma, fire;
-  const size_t need = gate_scratch(p, d, 0, &sigma, &fire);
+  ScoreScratch sc;
+  const size_t gate_end = gate_scratch(p, d, 0, &sigma, &fire);
+  const size_t need = centroid_tc(p) ? score_scratch(p, d, gate_end, &sc) : gate_end;
   if (need && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
                ws_bytes < need))
     return SBSA_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   SelectArgs a = select_args(p, d, q_cent, k_cent, p->rescue ? k_radius : nullptr, idx, cnt,
                              flags);
-  return run_select(p, d, a, static_cast<unsigned char*>(workspace), sigma, fire,
-                    static_cast<cudaStream_t>(stream));
+  if (centroid_tc(p)) {
+    float* scores = reinterpret_cast<float*>(ws + sc.scores);
+    rc = cuda_code(launch_centroid_scores(centroid_args(p, d, q_cent, k_cent, ws, sc, scores), s));
+    if (rc) return rc;
+    a.scores = scores;  // the pooled queries stay for the rescue bound
+  }
+  return run_select(p, d, a, ws, sigma, fire, s);
 }
 
 int sbsa_attend(const sbsa_params* p, const void* q, const void* k, const void* v,
@@ -436,12 +519,16 @@ int sbsa_prefill(const sbsa_params* p, const void* q, const void* k, const void*
   rc = cuda_code(launch_pool(p->dtype, d.ds, p->seq_len, p->block_size, jobs, rowmax ? 1 : 2, s));
   if (rc) return rc;
   SelectArgs sa = select_args(p, d, qc, kc, kr, idx, cnt, flags);
+  float* scores = reinterpret_cast<float*>(ws + w.sc.scores);
   if (p->tile_score == SBSA_TILE_ROWMAX) {
-    float* scores = reinterpret_cast<float*>(ws + w.scores);
-    rc = cuda_code(launch_rowmax(rowmax_args(p, d, xs_q, kc, ws + w.cbf, scores), s));
+    rc = cuda_code(launch_rowmax(rowmax_args(p, d, xs_q, kc, ws + w.sc.cbf, scores), s));
     if (rc) return rc;
     sa.scores = scores;
     sa.qc = nullptr;
+  } else if (centroid_tc(p)) {
+    rc = cuda_code(launch_centroid_scores(centroid_args(p, d, qc, kc, ws, w.sc, scores), s));
+    if (rc) return rc;
+    sa.scores = scores;  // the pooled queries stay for the rescue bound
   }
   rc = run_select(p, d, sa, ws, w.sigma, w.fire, s);
   if (rc) return rc;

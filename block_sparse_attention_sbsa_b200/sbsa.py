@@ -27,7 +27,9 @@ TILE_MEAN, TILE_ROWMAX = 0, 1
 FLAG_GATE, FLAG_RESCUE = 1, 2
 
 SYMBOLS = ["sbsa_pool_blocks", "sbsa_pool_minmax", "sbsa_select", "sbsa_select_ws",
-           "sbsa_select_workspace_bytes", "sbsa_score_rowmax", "sbsa_score_rowmax_workspace_bytes",
+           "sbsa_select_workspace_bytes", "sbsa_score_centroids",
+           "sbsa_score_centroids_workspace_bytes", "sbsa_score_rowmax",
+           "sbsa_score_rowmax_workspace_bytes",
            "sbsa_select_scores", "sbsa_attend", "sbsa_prefill",
            "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string",
            "sbsa_version", "sbsa_debug_wait_timeout"]
@@ -93,6 +95,9 @@ def _load() -> ctypes.CDLL:
     lib.sbsa_select_ws.argtypes = [P, f32p, f32p, f32p, i32p, i32p, u8p, vp, ctypes.c_size_t, vp]
     lib.sbsa_select_workspace_bytes.argtypes = [P]
     lib.sbsa_select_workspace_bytes.restype = ctypes.c_size_t
+    lib.sbsa_score_centroids.argtypes = [P, f32p, f32p, f32p, vp, ctypes.c_size_t, vp]
+    lib.sbsa_score_centroids_workspace_bytes.argtypes = [P]
+    lib.sbsa_score_centroids_workspace_bytes.restype = ctypes.c_size_t
     lib.sbsa_score_rowmax.argtypes = [P, vp, f32p, f32p, vp, ctypes.c_size_t, vp]
     lib.sbsa_score_rowmax_workspace_bytes.argtypes = [P]
     lib.sbsa_score_rowmax_workspace_bytes.restype = ctypes.c_size_t
@@ -232,10 +237,13 @@ def pool_minmax(p: Params, x: torch.Tensor, stream=None):
 
 
 def select(p: Params, q_cent: torch.Tensor, k_cent: torch.Tensor,
-           k_radius: Optional[torch.Tensor] = None, stream=None, with_flags: bool = True):
+           k_radius: Optional[torch.Tensor] = None, stream=None, with_flags: bool = True,
+           fma_scores: bool = False):
     """Block lists (idx [Hs, NB, Kmax], cnt [Hs, NB], flags [Hs, NB]).  k_cent
     is the centroid table [Hkv, NB, ds], or the min/max table [Hkv, NB, 2, ds]
-    of pool_minmax when p.backbone is BACKBONE_MINMAX."""
+    of pool_minmax when p.backbone is BACKBONE_MINMAX.  Calls sbsa_select_ws
+    (centroid scores on the tensor cores), or with fma_scores sbsa_select
+    (fp32 FMA scores inside the selection kernel; no percentile gate)."""
     nb, hs, ds = p.n_blocks, p.n_sel_heads, p.score_dim
     _need(q_cent, "q_cent", torch.float32, (hs, nb, ds))
     kshape = (p.n_kv_heads, nb, 2, ds) if p.backbone == BACKBONE_MINMAX else (p.n_kv_heads, nb, ds)
@@ -246,12 +254,32 @@ def select(p: Params, q_cent: torch.Tensor, k_cent: torch.Tensor,
     idx = torch.empty(hs, nb, p.max_blocks, device=dev, dtype=torch.int32)
     cnt = torch.empty(hs, nb, device=dev, dtype=torch.int32)
     flags = torch.empty(hs, nb, device=dev, dtype=torch.uint8) if with_flags else None
+    if fma_scores:
+        _check(lib.sbsa_select(ctypes.byref(p), _ptr(q_cent), _ptr(k_cent),
+                               _ptr(k_radius) if p.rescue else None, _ptr(idx), _ptr(cnt),
+                               _ptr(flags), _stream(stream)), "sbsa_select")
+        return idx, cnt, flags
     wsb = int(lib.sbsa_select_workspace_bytes(ctypes.byref(p)))
     ws = torch.empty(wsb, device=dev, dtype=torch.uint8) if wsb else None
     _check(lib.sbsa_select_ws(ctypes.byref(p), _ptr(q_cent), _ptr(k_cent),
                               _ptr(k_radius) if p.rescue else None, _ptr(idx), _ptr(cnt),
                               _ptr(flags), _ptr(ws), wsb, _stream(stream)), "sbsa_select_ws")
     return idx, cnt, flags
+
+
+def score_centroids(p: Params, q_cent: torch.Tensor, k_cent: torch.Tensor, stream=None):
+    """Centroid scores [Hs, NB, NB] on the tensor cores (entries j < i of row i
+    are defined, the rest stay 0)."""
+    nb, hs, ds = p.n_blocks, p.n_sel_heads, p.score_dim
+    _need(q_cent, "q_cent", torch.float32, (hs, nb, ds))
+    _need(k_cent, "k_cent", torch.float32, (p.n_kv_heads, nb, ds))
+    dev = q_cent.device
+    scores = torch.zeros(hs, nb, nb, device=dev, dtype=torch.float32)
+    wsb = int(lib.sbsa_score_centroids_workspace_bytes(ctypes.byref(p)))
+    ws = torch.empty(max(wsb, 1), device=dev, dtype=torch.uint8)
+    _check(lib.sbsa_score_centroids(ctypes.byref(p), _ptr(q_cent), _ptr(k_cent), _ptr(scores),
+                                    _ptr(ws), wsb, _stream(stream)), "sbsa_score_centroids")
+    return scores
 
 
 def score_rowmax(p: Params, q_src: torch.Tensor, k_cent: torch.Tensor, stream=None):

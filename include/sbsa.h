@@ -171,6 +171,27 @@ int sbsa_select(const sbsa_params* p, const float* q_cent, const float* k_cent,
  * sbsa_select_ws. */
 
 /*
+ * sbsa_score_centroids -- [UGS] step 1 / [RBS] base branch scores as one
+ * dense product on the tensor cores (mean backbone, mean tile scores).
+ *   q_cent   device fp32 [Hs, NB, ds] pooled queries (sbsa_pool_blocks).
+ *   k_cent   device fp32 [Hkv, NB, ds] key centroids.
+ *   scores   device fp32 [Hs, NB, NB] out: scores[hs, i, j] for j < i is
+ *            (q_cent[hs,i] . k_cent[g,j]) * score_scale, g as in sbsa_select;
+ *            entries j >= i are not written.
+ *   workspace device, 256-byte aligned, >= sbsa_score_centroids_workspace_bytes(p)
+ *            (tf32 hi / lo parts of both tables).
+ * Each product is taken as three tf32 products of the split operands
+ * (x = hi + lo), within a few fp32 roundings of the exact dot product; the
+ * summation order is the tensor core's.
+ * Errors as sbsa_select, plus SBSA_ERR_UNSUPPORTED unless p->backbone is
+ * SBSA_BACKBONE_MEAN and p->tile_score is SBSA_TILE_MEAN, and
+ * SBSA_ERR_WORKSPACE for a missing, misaligned or short workspace.
+ */
+size_t sbsa_score_centroids_workspace_bytes(const sbsa_params* p);
+int sbsa_score_centroids(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                         float* scores, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * sbsa_score_rowmax -- the page's tile scores (SBSA_TILE_ROWMAX).
  *   q_src    device [Hq, N, ds] bf16: Q, or Q_idx when p->index_dim is set.
  *   k_cent   device fp32 [Hkv, NB, ds] key centroids (sbsa_pool_blocks).
@@ -195,8 +216,9 @@ int sbsa_score_rowmax(const sbsa_params* p, const void* q_src, const float* k_ce
 int sbsa_select_scores(const sbsa_params* p, const float* scores, int32_t* idx, int32_t* cnt,
                        uint8_t* flags, void* workspace, size_t ws_bytes, void* stream);
 
-/* Device workspace sbsa_select_ws needs (0 when no gate needs one; also 0
- * when p is invalid). */
+/* Device workspace sbsa_select_ws needs: the percentile gate's scratch,
+ * and with the mean backbone and mean tile scores the score table and the
+ * scratch of sbsa_score_centroids.  0 when neither applies or p is invalid. */
 size_t sbsa_select_workspace_bytes(const sbsa_params* p);
 
 /*
@@ -204,7 +226,10 @@ size_t sbsa_select_workspace_bytes(const sbsa_params* p);
  * ws_bytes >= sbsa_select_workspace_bytes(p)) for the percentile gate's
  * per-row margins and per-tile decisions: three launches (top-k lists and
  * margins; the tile decisions; top-rho*k lists of the fired tiles).  The
- * pages have no entry point; the gate is theirs.
+ * pages have no entry point; the gate is theirs.  With the mean backbone and
+ * mean tile scores the scores come from sbsa_score_centroids into the
+ * workspace (tensor cores) instead of fp32 FMA inside the selection kernel,
+ * as they do in sbsa_prefill; sbsa_select keeps the FMA form.
  */
 int sbsa_select_ws(const sbsa_params* p, const float* q_cent, const float* k_cent,
                    const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,

@@ -88,6 +88,18 @@ def _valid(sb, **kw):
 FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced on the host
 
 
+def r256(x):
+    return (x + 255) // 256 * 256
+
+
+def _centroid_scratch(p, with_table=True):
+    """Bytes of the tensor-core centroid scores' scratch: tf32 hi and lo parts
+    of the pooled queries and of the centroids, then the [Hs, NB, NB] table."""
+    nb, hs, ds = p.n_blocks, p.n_sel_heads, p.score_dim
+    parts = 2 * r256(hs * nb * ds * 4) + 2 * r256(p.n_kv_heads * nb * ds * 4)
+    return parts + (r256(hs * nb * nb * 4) if with_table else 0)
+
+
 def _select(sb, p):
     return sb.lib.sbsa_select(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, None)
 
@@ -166,27 +178,49 @@ def test_minmax_backbone_doubles_the_key_table_in_the_workspace(sb):
     mean = _valid(sb)
     mm = _valid(sb, backbone="minmax")
     nb = mean.n_blocks
-
-    def r256(x):
-        return (x + 255) // 256 * 256
     extra = r256(2 * 2 * nb * 128 * 4) - r256(2 * nb * 128 * 4)
-    assert sb.workspace_bytes(mm) == sb.workspace_bytes(mean) + extra
+    # the upper bound is no product: no tensor-core score scratch
+    assert sb.workspace_bytes(mm) == sb.workspace_bytes(mean) - _centroid_scratch(mean) + extra
+
+
+def test_centroid_scores_workspace_and_checks(sb):
+    p = _valid(sb, seq_len=4096)
+    need = sb.lib.sbsa_score_centroids_workspace_bytes(ctypes.byref(p))
+    assert need == _centroid_scratch(p, with_table=False)
+    for other in (_valid(sb, backbone="minmax"), _valid(sb, tile_score="rowmax")):
+        assert sb.lib.sbsa_score_centroids_workspace_bytes(ctypes.byref(other)) == 0
+        assert sb.lib.sbsa_score_centroids(ctypes.byref(other), FAKE, FAKE, FAKE, FAKE, need,
+                                           None) == 2
+    f = sb.lib.sbsa_score_centroids
+    assert f(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, need - 1, None) == 3
+    assert f(ctypes.byref(p), FAKE, FAKE, FAKE, ctypes.c_void_p((1 << 20) + 128), need, None) == 3
+    assert f(ctypes.byref(p), None, FAKE, FAKE, FAKE, need, None) == 1
+    assert f(ctypes.byref(p), FAKE, FAKE, ctypes.c_void_p((1 << 20) + 4), FAKE, need, None) == 1
+    # sbsa_select_ws needs the table and its scratch; sbsa_select none
+    assert sb.lib.sbsa_select_workspace_bytes(ctypes.byref(p)) == _centroid_scratch(p)
+    ws = sb.lib.sbsa_select_ws
+    assert ws(ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, None, FAKE,
+              _centroid_scratch(p) - 1, None) == 3
+    assert ws(ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, None, None, 0, None) == 3
 
 
 def test_percentile_gate_needs_a_workspace(sb):
     p = _valid(sb, gate_quantile=0.3, gate_rho=2, seq_len=4096)
     nb = p.n_blocks
     need = sb.lib.sbsa_select_workspace_bytes(ctypes.byref(p))
-    assert need == (4 * nb * 8 + 255) // 256 * 256 + (nb + 255) // 256 * 256
-    assert sb.lib.sbsa_select_workspace_bytes(ctypes.byref(_valid(sb))) == 0
+    gate = (4 * nb * 8 + 255) // 256 * 256 + (nb + 255) // 256 * 256
+    assert need == gate + _centroid_scratch(p)
+    mm = _valid(sb, gate_quantile=0.3, gate_rho=2, seq_len=4096, backbone="minmax")
+    assert sb.lib.sbsa_select_workspace_bytes(ctypes.byref(mm)) == gate
+    assert sb.lib.sbsa_select_workspace_bytes(ctypes.byref(_valid(sb, backbone="minmax"))) == 0
     assert _select(sb, p) == 3                   # the plain entry point has no workspace
     ws = sb.lib.sbsa_select_ws
     assert ws(ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, None, FAKE, need - 1, None) == 3
     assert ws(ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, None,
               ctypes.c_void_p((1 << 20) + 64), need, None) == 3
-    # the prefill workspace grows by the same scratch
+    # the prefill workspace grows by the gate's scratch
     plain = sb.workspace_bytes(_valid(sb, seq_len=4096, max_blocks=p.max_blocks))
-    assert sb.workspace_bytes(p) == plain + need
+    assert sb.workspace_bytes(p) == plain + gate
 
 
 def test_rowmax_workspace_and_checks(sb):
@@ -199,10 +233,12 @@ def test_rowmax_workspace_and_checks(sb):
     assert f(ctypes.byref(_valid(sb)), FAKE, FAKE, FAKE, FAKE, need, None) == 2  # not rowmax
     assert f(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, need - 1, None) == 3
     assert f(ctypes.byref(p), None, FAKE, FAKE, FAKE, need, None) == 1
-    # the prefill workspace holds the bf16 centroids and the score table too
-    plain = sb.workspace_bytes(_valid(sb, seq_len=4096))
+    # the prefill workspace holds the bf16 centroids and the score table
+    # in place of the tensor-core centroid scratch
+    mean = _valid(sb, seq_len=4096)
+    plain = sb.workspace_bytes(mean) - _centroid_scratch(mean)
     scores = (4 * nb * nb * 4 + 255) // 256 * 256
-    assert sb.workspace_bytes(p) >= plain + need + scores - 256
+    assert sb.workspace_bytes(p) == plain + need + scores
 
 
 def test_fp32_attention_is_limited_to_d64_b64(sb):
@@ -214,11 +250,9 @@ def test_workspace_size_and_checks(sb):
     p = _valid(sb, rescue_tau=5.0)
     nb = p.n_blocks
     ws = sb.workspace_bytes(p)
-
-    def r256(x):
-        return (x + 255) // 256 * 256
     want = (r256(4 * nb * 128 * 4) + r256(2 * nb * 128 * 4) + r256(2 * nb * 4)
-            + r256(4 * nb * p.max_blocks * 4) + r256(4 * nb * 4) + r256(4 * nb))
+            + r256(4 * nb * p.max_blocks * 4) + r256(4 * nb * 4) + r256(4 * nb)
+            + _centroid_scratch(p))
     assert ws == want
     small = sb.lib.sbsa_prefill(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
                                 ws - 1, None, None, None, None)

@@ -109,10 +109,48 @@ def test_pool_matches_oracle(sb, name):
     assert sb.get_status() == sb.OK
 
 
-@pytest.mark.parametrize("name", SMALL_NAMES)
-def test_select_on_oracle_tables(sb, name):
-    """Selection alone: the oracle's pooled tables in, lists out."""
+MEAN_NAMES = [n for n in SMALL_NAMES
+              if W.SMALL[n].backbone == "mean" and W.SMALL[n].tile_score == "mean"]
+
+
+@pytest.mark.parametrize("name", MEAN_NAMES)
+def test_centroid_scores_match_oracle(sb, name):
+    """The tensor-core centroid scores (three tf32 products per pair) against
+    the exact dot products of the same fp32 tables, for every (selection
+    head, tile i, j < i); entries j >= i stay unwritten."""
     w, data, ref = small_case(name)
+    p = sb.params_for(w)
+    qc32 = np.asarray(ref["qbar"], dtype=np.float32)
+    kc32 = np.asarray(ref["c"], dtype=np.float32)
+    got = sb.score_centroids(p, torch.tensor(qc32, device="cuda"),
+                             torch.tensor(kc32, device="cuda")).cpu().numpy()
+    assert sb.get_status() == sb.OK
+    scale = float(np.float32(1.0) / np.sqrt(np.float32(w.score_dim)))
+    kv = _kv_of_sel(w)
+    for hs in range(w.n_sel_heads):
+        q = qc32[hs].astype(np.float64)
+        c = kc32[kv(hs)].astype(np.float64)
+        want = (q @ c.T) * scale               # [i, j], exact products of the inputs
+        mag = (np.abs(q) @ np.abs(c).T) * scale
+        for i in range(w.n_blocks):
+            err = np.abs(got[hs, i, :i] - want[i, :i])
+            # three tf32 products keep each term within 3 * 2^-20 of x*y; the
+            # rest is fp32 accumulation and the final rounding
+            tol = 2.0 ** -16 * mag[i, :i] + 2.0 ** -23 * np.abs(want[i, :i])
+            # (a dropped hi*lo product would leave errors near 2^-11 of it)
+            assert np.all(err <= tol), (hs, i, float((err - tol).max()))
+            assert np.all(got[hs, i, i:] == 0.0)
+
+
+@pytest.mark.parametrize("name", SMALL_NAMES)
+@pytest.mark.parametrize("path", ["tensor", "fma"])
+def test_select_on_oracle_tables(sb, name, path):
+    """Selection alone: the oracle's pooled tables in, lists out.  "tensor":
+    sbsa_select_ws (centroid scores on the tensor cores where they apply);
+    "fma": sbsa_select (fp32 FMA scores inside the selection kernel)."""
+    w, data, ref = small_case(name)
+    if path == "fma" and (w.tile_score == "rowmax" or w.gate_quantile is not None):
+        pytest.skip("sbsa_select has no workspace for the percentile gate or tile scores")
     p = sb.params_for(w)
     qc = torch.tensor(ref["qbar"], dtype=torch.float32, device="cuda")
     if w.backbone == "minmax":
@@ -129,7 +167,8 @@ def test_select_on_oracle_tables(sb, name):
                 table[hs, i, :i] = fn(hs, i)
         idx, cnt, flags = sb.select_scores(p, torch.tensor(table, device="cuda"))
     else:
-        idx, cnt, flags = sb.select(p, qc, kc, kr if w.rescue_tau is not None else None)
+        idx, cnt, flags = sb.select(p, qc, kc, kr if w.rescue_tau is not None else None,
+                                    fma_scores=path == "fma")
     idx, cnt, flags = idx.cpu().numpy(), cnt.cpu().numpy(), flags.cpu().numpy()
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
                                   ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"],
