@@ -18,15 +18,19 @@
 // sum_d max(q_d min_d, q_d max_d) over the block's coordinate box.
 //
 // Layout of one CTA: R (up to 16) consecutive query blocks of one selection
-// head.  Phase 1 computes their scores against every earlier key block into
-// shared memory: each thread streams whole key-centroid rows from L2 in
-// 16-byte pieces and dots them with the R pooled queries held in shared
-// memory (fp32 FMA; each centroid row is read once per CTA).  Phase 2 gives
-// each row to a warp:
-// exact radix selection on order-preserving 32-bit keys (ties resolved by the
-// lower block id), 64-bit fixed-point mass histograms for the cumulative-mass
-// rule (deterministic sums), double-precision mean/std for the gate, then a
-// ballot compaction that emits the ascending list.
+// head.  Phase 1 puts their scores against every earlier key block into
+// shared memory: copied from a precomputed table (the tensor-core centroid
+// scores, or the row-max tile scores), or computed here -- each thread
+// streams whole key-centroid rows from L2 in 16-byte pieces and dots them
+// with the R pooled queries held in shared memory (fp32 FMA; each centroid
+// row is read once per CTA).  The kv head's block radii are staged beside
+// them for the rescue branch.  Phase 2 gives each row to a warp: exact radix
+// selection on order-preserving 32-bit keys (ties resolved by the lower
+// block id), a ranked walk with 64-bit fixed-point masses for the
+// cumulative-mass rule (radix selection on mass histograms past 24 blocks;
+// deterministic sums), double-precision mean/std for the gate, then a ballot
+// compaction that emits the ascending list.  The scans keep four 32-wide
+// chunks in flight per warp.
 #include <cstdint>
 
 #include "internal.h"
@@ -294,6 +298,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
   float* qs = reinterpret_cast<float*>(smem_raw);                 // [R][DS]
   unsigned char* hist_base = reinterpret_cast<unsigned char*>(qs + R * DS);  // phase 2
   float* sc = reinterpret_cast<float*>(hist_base + kHistBytes);   // [R][score_stride]
+  float* krs = sc + (size_t)R * score_stride;                     // [score_stride] radii (rescue)
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -316,6 +321,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
     const int r = e / DS;
     qs[e] = (r < rows && a.qc) ? a.qc[((size_t)hs * a.nb + i0 + r) * DS + (e % DS)] : 0.f;
   }
+  if (a.rescue) {
+    // the kv head's radii of every candidate, read once per CTA
+    const float* kr = a.kr + (size_t)g * a.nb;
+    for (int j = tid; j < jend; j += kSelThreads) krs[j] = kr[j];
+  }
   __syncthreads();
 
   // ---- phase 1: scores.  Each thread owns candidate blocks j = tid + 256u
@@ -323,10 +333,33 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
   // each piece with the R pooled queries read from shared memory (every lane
   // reads the same address: one broadcast per row).
   if (a.scores) {
-    // precomputed tile scores (row-max): copy the rows' candidates
-    for (int r = 0; r < rows; ++r) {
-      const float* src = a.scores + ((size_t)hs * a.nb + i0 + r) * a.nb;
-      for (int j = tid; j < i0 + r; j += kSelThreads) sc[r * score_stride + j] = src[j];
+    // precomputed scores (centroid or row-max): copy the rows' candidates,
+    // four rows' loads in flight per thread
+    const float* base = a.scores + ((size_t)hs * a.nb + i0) * a.nb;
+    if ((a.nb & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0) {
+      for (int r0 = 0; r0 < rows; r0 += 4) {
+        for (int j4 = tid; 4 * j4 < i0 + r0 + 3; j4 += kSelThreads) {
+          float4 v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u;
+            v[u] = (r < rows && 4 * j4 < i0 + r)
+                       ? __ldg(reinterpret_cast<const float4*>(base + (size_t)r * a.nb) + j4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u;
+            if (r < rows && 4 * j4 < i0 + r)
+              *reinterpret_cast<float4*>(sc + r * score_stride + 4 * j4) = v[u];
+          }
+        }
+      }
+    } else {
+      for (int r = 0; r < rows; ++r) {
+        const float* src = base + (size_t)r * a.nb;
+        for (int j = tid; j < i0 + r; j += kSelThreads) sc[r * score_stride + j] = src[j];
+      }
     }
   } else if (a.minmax) {
     // Upper-bound backbone: s_j = sum_d max(q_d min_jd, q_d max_jd), the two
@@ -478,12 +511,23 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
       if (n == 0) {
         select_all = true;
       } else {
-        float m = -INFINITY;
-        for (int j = lane; j < n; j += 32) m = fmaxf(m, s[j]);
-        m = warp_max_f(m);
-        double z = 0.0;
-        for (int j = lane; j < n; j += 32) z += (double)__expf(s[j] - m);
-        z = warp_sum_d(z);
+        // four independent partials per lane keep four loads in flight
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        int j = lane;
+        for (; j + 96 < n; j += 128) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) m4[u] = fmaxf(m4[u], s[j + 32 * u]);
+        }
+        for (; j < n; j += 32) m4[0] = fmaxf(m4[0], s[j]);
+        const float m = warp_max_f(fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+        double z4[4] = {0.0, 0.0, 0.0, 0.0};
+        j = lane;
+        for (; j + 96 < n; j += 128) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) z4[u] += (double)__expf(s[j + 32 * u] - m);
+        }
+        for (; j < n; j += 32) z4[0] += (double)__expf(s[j] - m);
+        const double z = warp_sum_d((z4[0] + z4[1]) + (z4[2] + z4[3]));
         const double wscale = 1152921504606846976.0 / z;  // 2^60 / Z
         const uint64_t want = (uint64_t)ceil((double)a.mass * 1152921504606846976.0);
         // The kept prefix is usually a handful of blocks: walk the ranked
@@ -492,12 +536,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
         uint64_t prev = ~0ull, cum = 0;
         int taken = 0;
         for (; taken < kMaxWalk && taken < n; ++taken) {
-          uint64_t best = 0;
-          for (int j = lane; j < n; j += 32) {
-            const uint64_t c = rank_key(s[j], j);
-            if (c < prev && c > best) best = c;
+          uint64_t b4[4] = {0, 0, 0, 0};
+          int jj = lane;
+          for (; jj + 96 < n; jj += 128) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint64_t c = rank_key(s[jj + 32 * u], jj + 32 * u);
+              if (c < prev && c > b4[u]) b4[u] = c;
+            }
           }
-          best = warp_max_u64(best);
+          for (; jj < n; jj += 32) {
+            const uint64_t c = rank_key(s[jj], jj);
+            if (c < prev && c > b4[0]) b4[0] = c;
+          }
+          const uint64_t b01 = b4[0] > b4[1] ? b4[0] : b4[1];
+          const uint64_t b23 = b4[2] > b4[3] ? b4[2] : b4[3];
+          const uint64_t best = warp_max_u64(b01 > b23 ? b01 : b23);
           prev = best;
           cum += mass_weight(key_float((uint32_t)(best >> 32)), m, wscale);
           if (cum >= want) {
@@ -543,41 +597,47 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
       for (int o = 16; o > 0; o >>= 1) q2 += __shfl_xor_sync(0xFFFFFFFFu, q2, o);
       qn_s = sqrtf(q2) * a.score_scale;
     }
-    const float* kr = a.rescue ? a.kr + (size_t)g * a.nb : nullptr;
-
     // ---- compaction: ascending ids, then the diagonal, then -1 ----
+    // The decisions of four 32-wide chunks are taken first (independent
+    // loads), then the chunks are emitted in order.
     int written = 0, tie_seen = 0;
     bool rescued_extra = false;
-    for (int base = 0; base < n; base += 32) {
-      const int j = base + lane;
-      const bool in = j < n;
-      bool sel = false, eqk = false, basesel = false;
-      if (in) {
-        if (select_all) {
-          basesel = true;
-        } else if (walked) {
-          basesel = rank_key(s[j], j) >= wkey;
-        } else {
-          const uint32_t u = fkey(s[j]);
-          basesel = u > vkey;
-          eqk = (u == vkey);
+    for (int base = 0; base < n; base += 128) {
+      bool bsel[4], eqk[4], resc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = base + 32 * u + lane;
+        bsel[u] = false;
+        eqk[u] = false;
+        resc[u] = false;
+        if (j < n) {
+          const float sj = s[j];
+          if (select_all) {
+            bsel[u] = true;
+          } else if (walked) {
+            bsel[u] = rank_key(sj, j) >= wkey;
+          } else {
+            const uint32_t k = fkey(sj);
+            bsel[u] = k > vkey;
+            eqk[u] = k == vkey;
+          }
+          if (a.rescue) resc[u] = fmaf(qn_s, krs[j], sj) > a.tau;
         }
       }
-      const unsigned eqmask = __ballot_sync(0xFFFFFFFFu, eqk);
-      if (eqk) basesel = (tie_seen + __popc(eqmask & lt_mask)) < take_eq;
-      tie_seen += __popc(eqmask);
-      sel = basesel;
-      if (in && a.rescue) {
-        const float ub = fmaf(qn_s, kr[j], s[j]);
-        if (ub > a.tau) {
-          sel = true;
-          if (!basesel) rescued_extra = true;
-        }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (base + 32 * u >= n) break;  // uniform over the warp
+        const unsigned eqmask = __ballot_sync(0xFFFFFFFFu, eqk[u]);
+        bool basesel = bsel[u];
+        if (eqk[u]) basesel = (tie_seen + __popc(eqmask & lt_mask)) < take_eq;
+        tie_seen += __popc(eqmask);
+        const bool sel = basesel || resc[u];
+        if (resc[u] && !basesel) rescued_extra = true;
+        const unsigned selmask = __ballot_sync(0xFFFFFFFFu, sel);
+        const int pos = written + __popc(selmask & lt_mask);
+        if (sel && pos < a.kmax - 1) out[pos] = base + 32 * u + lane;
+        written += __popc(selmask);
       }
-      const unsigned selmask = __ballot_sync(0xFFFFFFFFu, sel);
-      const int pos = written + __popc(selmask & lt_mask);
-      if (sel && pos < a.kmax - 1) out[pos] = j;
-      written += __popc(selmask);
     }
     if (__any_sync(0xFFFFFFFFu, rescued_extra)) flag |= 2;
     if (written > a.kmax - 1) {
@@ -589,7 +649,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
       a.cnt[(size_t)hs * a.nb + i] = written + 1;
       if (a.flags) a.flags[(size_t)hs * a.nb + i] = flag;
     }
-    for (int p = written + 1 + lane; p < a.kmax; p += 32) out[p] = -1;
+    // -1 padding, 16 bytes per store once the row position is aligned
+    int p = written + 1;
+    const int head = min(a.kmax, (p + 3) & ~3);
+    if (p + lane < head) out[p + lane] = -1;
+    p = head;
+    if ((reinterpret_cast<uintptr_t>(out + p) & 15) == 0) {
+      const int n4 = (a.kmax - p) >> 2;
+      int4* o4 = reinterpret_cast<int4*>(out + p);
+      for (int q = lane; q < n4; q += 32) o4[q] = make_int4(-1, -1, -1, -1);
+      p += 4 * n4;
+    }
+    for (int q = p + lane; q < a.kmax; q += 32) out[q] = -1;
     __syncwarp();
   }
 }
@@ -597,7 +668,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
 template <int DS, int R>
 cudaError_t launch_rows(const SelectArgs& a, cudaStream_t stream) {
   const int stride = (a.nb + 3) & ~3;
-  const size_t smem = (size_t)R * DS * 4 + kHistBytes + (size_t)R * stride * 4;
+  const size_t smem = (size_t)R * DS * 4 + kHistBytes + (size_t)R * stride * 4 +
+                      (a.rescue ? (size_t)stride * 4 : 0);
   auto kern = select_kernel<DS, R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -645,10 +717,11 @@ cudaError_t launch_ds(const SelectArgs& a, cudaStream_t stream) {
   // more rows per CTA means fewer reads of each centroid row from L2
   const size_t budget = 200 * 1024;
   const size_t row = (size_t)((a.nb + 3) & ~3) * 4 + DS * 4;
-  if (kHistBytes + 16 * row <= budget) return launch_rows<DS, 16>(a, stream);
-  if (kHistBytes + 8 * row <= budget) return launch_rows<DS, 8>(a, stream);
-  if (kHistBytes + 4 * row <= budget) return launch_rows<DS, 4>(a, stream);
-  if (kHistBytes + 2 * row <= budget) return launch_rows<DS, 2>(a, stream);
+  const size_t fixed = kHistBytes + (a.rescue ? (size_t)((a.nb + 3) & ~3) * 4 : 0);
+  if (fixed + 16 * row <= budget) return launch_rows<DS, 16>(a, stream);
+  if (fixed + 8 * row <= budget) return launch_rows<DS, 8>(a, stream);
+  if (fixed + 4 * row <= budget) return launch_rows<DS, 4>(a, stream);
+  if (fixed + 2 * row <= budget) return launch_rows<DS, 2>(a, stream);
   return cudaErrorInvalidValue;
 }
 
