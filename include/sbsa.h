@@ -209,9 +209,17 @@ int sbsa_score_rowmax(const sbsa_params* p, const void* q_src, const float* k_ce
                       float* scores, void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * sbsa_select_scores -- sbsa_select_ws on precomputed tile scores
- * [Hs, NB, NB] (sbsa_score_rowmax) instead of pooled tables; every rule
- * (top-k, the gates, cumulative mass, the diagonal) applies unchanged.
+ * sbsa_select_scores -- the selection on a precomputed score table
+ * [Hs, NB, NB] (sbsa_score_rowmax or sbsa_score_centroids; row i holds the
+ * scores of candidates j < i, the rest is not read) instead of pooled
+ * tables; every rule (top-k, the gates, cumulative mass, the diagonal)
+ * applies unchanged.  Outputs as sbsa_select.
+ *   workspace  used only by the percentile gate (its per-row margins and
+ *              per-tile decisions); a workspace of sbsa_select_workspace_bytes(p)
+ *              bytes, 256-byte aligned, always suffices.
+ * Errors as sbsa_select; SBSA_ERR_INVALID_ARG with p->rescue (the rescue bound
+ * needs the pooled tables); SBSA_ERR_WORKSPACE for a missing or short
+ * workspace under the percentile gate.
  */
 int sbsa_select_scores(const sbsa_params* p, const float* scores, int32_t* idx, int32_t* cnt,
                        uint8_t* flags, void* workspace, size_t ws_bytes, void* stream);
