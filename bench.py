@@ -38,7 +38,7 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention launch, from the
 # ncu capture summarised in profiles/ (None until captured for this kernel).
-NCU_ATTEND_TRAFFIC = {"rbs128k": 5.62e9 + 1.05e9}
+NCU_ATTEND_TRAFFIC = {"rbs128k": 5.608e9 + 1.050e9}
 
 
 def selection_stats(w, p, st, meta) -> dict:
