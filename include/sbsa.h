@@ -256,8 +256,9 @@ int sbsa_attend(const sbsa_params* p, const void* q, const void* k, const void* 
                 const int32_t* idx, const int32_t* cnt, void* o, void* stream);
 
 /* Bytes of device workspace sbsa_prefill needs for these parameters
- * (pooled tables, plus lists when the caller does not provide them).
- * Returns 0 when p is invalid. */
+ * (pooled tables; the score table with its scratch for the mean backbone
+ * and for row-max tile scores; the percentile gate's scratch; plus lists when
+ * the caller does not provide them).  Returns 0 when p is invalid. */
 size_t sbsa_prefill_workspace_bytes(const sbsa_params* p);
 
 /*
@@ -305,8 +306,9 @@ int sbsa_debug_wait_timeout(uint64_t timeout_ns, void* stream);
  * allocator, a latency-critical path where cudaMalloc's implicit device
  * synchronisation is not acceptable, or a process whose device memory
  * budget is fixed at start-up.  This entry point takes the same inputs and
- * outputs as sbsa_prefill minus the workspace; its temporaries (pooled
- * tables and, when idx_out/cnt_out are NULL, the block lists) live in one
+ * outputs as sbsa_prefill minus the workspace; its temporaries (those of
+ * sbsa_prefill_workspace_bytes: pooled tables, score table and scratch and,
+ * when idx_out/cnt_out are NULL, the block lists) live in one
  * fixed array of SBSA_NOALLOC_SCRATCH_BYTES compiled into the library.  It
  * calls no cudaMalloc, cudaFree or other allocating routine.
  *
