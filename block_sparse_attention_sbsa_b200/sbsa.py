@@ -392,9 +392,11 @@ def get_status(stream=None) -> int:
 class Staged:
     """The prefill as its separate C-ABI stages on preallocated buffers:
     pool keys (centroids + radii, or the min/max table of the upper-bound
-    backbone), pool queries, select, attend.  Each method is one library call
-    and allocates nothing; the kernels are the ones sbsa_prefill launches
-    (which merges the two pooling jobs into one grid)."""
+    backbone), pool queries (or the row-max tile scores), select (with the
+    mean backbone: tf32 split, tensor-core centroid scores, selection), attend.
+    Each method is one or two library calls and allocates nothing; the kernels
+    are the ones sbsa_prefill launches (which merges the two pooling jobs into
+    one grid)."""
 
     def __init__(self, p: Params, device="cuda"):
         self.p = p
