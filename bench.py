@@ -156,14 +156,24 @@ class ClockSampler:
         self.tmp = None
 
     def start(self):
+        """Start sampling every 20 ms and return once the first sample is in,
+        so that even a timed region of a few tens of milliseconds is sampled
+        (the first sample, taken just before the region, is dropped when
+        later ones exist)."""
         try:
             self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.tmp, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        deadline = time.time() + 3.0
+        while time.time() < deadline and self.proc.poll() is None:
+            if os.path.getsize(self.tmp.name) > 0:
+                break
+            time.sleep(0.005)
 
     def stop(self):
         if self.proc is None:
@@ -179,9 +189,10 @@ class ClockSampler:
         os.unlink(self.tmp.name)
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = [r for r in rows if len(r) >= 9]
+        if len(rows) > 1:
+            rows = rows[1:]  # the first sample precedes the timed region
         for r in rows:
-            if len(r) < 9:
-                continue
             try:
                 sm.append(float(r[1]))
                 mx = float(r[2])
