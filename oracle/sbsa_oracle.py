@@ -170,20 +170,15 @@ def block_bounds_minmax(qbar_i, kmin_g, kmax_g, i: int, scale: float):
     return (np.maximum(lo, hi).sum(axis=1) * scale).astype(np.float32)
 
 
-def bf16_round(x) -> np.ndarray:
-    """Round-to-nearest-even to bfloat16, returned as float64."""
-    f = np.asarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32).astype(np.float64)
-
-
 def block_scores_rowmax(q_rows, c_g, i: int, scale: float):
     """Tile score of query block i against candidates j < i: the largest
-    q_t . bf16(c_j) over the tile's query rows t (all rows given, e.g. the
-    rows of every head of a group), times scale, rounded to float32."""
+    q_t . c_j over the tile's query rows t (all rows given, e.g. the rows of
+    every head of a group), times scale, in float64 from the centroids as
+    given, rounded to float32 once at the end (the precision the selection
+    decision is taken in).  The page defines the tile score as the largest
+    row score; nothing in it rounds the operands."""
     q = _f64(q_rows)
-    c = bf16_round(c_g[:i])
+    c = _f64(c_g[:i])
     if i == 0:
         return np.zeros(0, dtype=np.float32)
     return ((q @ c.T).max(axis=0) * scale).astype(np.float32)

@@ -26,3 +26,20 @@ def cuda():
     if not cuda_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_terminal_summary(terminalreporter):
+    """One line per parity check: rows compared, rows equal to the oracle's,
+    rows that differ only inside the fp32 tie band, percentile-gate tiles
+    inside their band, and output errors against the oracle."""
+    try:
+        import parity
+    except Exception:
+        return
+    if not parity.REPORT:
+        return
+    terminalreporter.write_sep("-", "parity against the oracle (tie band counted)")
+    for r in parity.REPORT:
+        rest = " ".join(f"{k}={v:.3g}" if isinstance(v, float) else f"{k}={v}"
+                        for k, v in r.items() if k not in ("test", "workload"))
+        terminalreporter.write_line(f"PARITY {r['test']} {r['workload']} {rest}")

@@ -41,6 +41,21 @@ def percentile_budgets(sbar: dict, fired: set, k: int, rho: int) -> dict:
     return out
 
 
+# Counts each parity test reports (printed in the session summary, see
+# conftest.py): exact and tie-band rows, tiles inside SIGMA_BAND, output errors.
+REPORT: list = []
+
+
+def record(test: str, workload: str, **counts) -> None:
+    REPORT.append(dict(test=test, workload=workload, **counts))
+
+
+def sigma_band_tiles(budgets) -> int:
+    """Tiles whose percentile-gate decision lies inside SIGMA_BAND of the cut
+    (either budget accepted)."""
+    return 0 if budgets is None else sum(1 for b in budgets.values() if len(b) > 1)
+
+
 def band(x: float) -> float:
     return BAND * max(1.0, abs(x))
 

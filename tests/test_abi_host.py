@@ -78,9 +78,13 @@ def test_status_strings(sb):
     assert sb.lib.sbsa_version() >= 100
 
 
-def _valid(sb, **kw):
-    base = dict(n_q_heads=4, n_kv_heads=2, seq_len=1000, head_dim=128, block_size=128,
+def _valid_base():
+    return dict(n_q_heads=4, n_kv_heads=2, seq_len=1000, head_dim=128, block_size=128,
                 dtype="bf16", select_mode="topk", top_k=4)
+
+
+def _valid(sb, **kw):
+    base = _valid_base()
     base.update(kw)
     return sb.make_params(**base)
 
@@ -227,18 +231,37 @@ def test_rowmax_workspace_and_checks(sb):
     p = _valid(sb, tile_score="rowmax", seq_len=4096)
     nb = p.n_blocks
     need = sb.lib.sbsa_score_rowmax_workspace_bytes(ctypes.byref(p))
-    assert need == (2 * nb * 128 * 2 + 255) // 256 * 256
+    assert need == (3 * 2 * nb * 128 * 2 + 255) // 256 * 256   # three bf16 parts
     assert sb.lib.sbsa_score_rowmax_workspace_bytes(ctypes.byref(_valid(sb))) == 0
     f = sb.lib.sbsa_score_rowmax
     assert f(ctypes.byref(_valid(sb)), FAKE, FAKE, FAKE, FAKE, need, None) == 2  # not rowmax
     assert f(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, need - 1, None) == 3
     assert f(ctypes.byref(p), None, FAKE, FAKE, FAKE, need, None) == 1
-    # the prefill workspace holds the bf16 centroids and the score table
+    # the prefill workspace holds the centroid parts and the score table
     # in place of the tensor-core centroid scratch
     mean = _valid(sb, seq_len=4096)
     plain = sb.workspace_bytes(mean) - _centroid_scratch(mean)
     scores = (4 * nb * nb * 4 + 255) // 256 * 256
     assert sb.workspace_bytes(p) == plain + need + scores
+
+
+@pytest.mark.parametrize("kw,ok_len,bad_len", [
+    # the selection kernel keeps two score rows of NB candidates in shared memory
+    (dict(top_k=4), 23424 * 128, 23425 * 128),
+    (dict(select_mode="cummass", mass_threshold=0.9, rescue_tau=5.0), 15616 * 128,
+     15617 * 128),
+    # the row-max kernel keeps the running maxima of a tile's candidates
+    (dict(top_k=4, tile_score="rowmax"), 16897 * 128, 16898 * 128),
+])
+def test_shared_memory_limits_are_rejected_before_launch(sb, kw, ok_len, bad_len):
+    base = dict(_valid_base(), **kw)
+    good = sb.make_params(**dict(base, seq_len=ok_len))
+    bad = sb.make_params(**dict(base, seq_len=bad_len))
+    assert sb.lib.sbsa_prefill_workspace_bytes(ctypes.byref(good)) > 0
+    assert sb.lib.sbsa_prefill_workspace_bytes(ctypes.byref(bad)) == 0
+    assert _select(sb, bad) == 2
+    assert sb.lib.sbsa_prefill(ctypes.byref(bad), FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
+                               1 << 40, None, None, None, None) == 2
 
 
 def test_fp32_attention_is_limited_to_d64_b64(sb):

@@ -127,6 +127,7 @@ def test_centroid_scores_match_oracle(sb, name):
     assert sb.get_status() == sb.OK
     scale = float(np.float32(1.0) / np.sqrt(np.float32(w.score_dim)))
     kv = _kv_of_sel(w)
+    worst = 0.0
     for hs in range(w.n_sel_heads):
         q = qc32[hs].astype(np.float64)
         c = kc32[kv(hs)].astype(np.float64)
@@ -140,6 +141,9 @@ def test_centroid_scores_match_oracle(sb, name):
             # (a dropped hi*lo product would leave errors near 2^-11 of it)
             assert np.all(err <= tol), (hs, i, float((err - tol).max()))
             assert np.all(got[hs, i, i:] == 0.0)
+            if i > 0:
+                worst = max(worst, float((err / np.maximum(1.0, np.abs(want[i, :i]))).max()))
+    PT.record("centroid_scores", name, worst_rel_err=worst, band=PT.BAND)
 
 
 @pytest.mark.parametrize("name", SMALL_NAMES)
@@ -170,9 +174,12 @@ def test_select_on_oracle_tables(sb, name, path):
         idx, cnt, flags = sb.select(p, qc, kc, kr if w.rescue_tau is not None else None,
                                     fma_scores=path == "fma")
     idx, cnt, flags = idx.cpu().numpy(), cnt.cpu().numpy(), flags.cpu().numpy()
+    budgets = _budgets(w, ref)
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
                                   ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"],
-                                  budgets=_budgets(w, ref), score_fn=_small_rowmax_fn(w, data, ref))
+                                  budgets=budgets, score_fn=_small_rowmax_fn(w, data, ref))
+    PT.record(f"select[{path}]", name, rows=exact + tie, exact=exact, tie=tie,
+              sigma_band_tiles=PT.sigma_band_tiles(budgets))
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # padding and flags
     for hs in range(w.n_sel_heads):
@@ -194,6 +201,7 @@ def test_attend_on_oracle_lists(sb, name):
     o = sb.attend(p, d["q"], d["k"], d["v"], idx, cnt)
     torch.cuda.synchronize()
     mx, mean = PT.output_errors(o.float().cpu().numpy(), ref["o"])
+    PT.record("attend", name, max_abs=mx, mean_abs=mean)
     assert sb.get_status() == sb.OK
     assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
 
@@ -207,9 +215,10 @@ def test_prefill_end_to_end(sb, name):
     torch.cuda.synchronize()
     assert sb.get_status() == sb.OK
     idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    budgets = _budgets(w, ref)
     exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
                                   ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"],
-                                  budgets=_budgets(w, ref), score_fn=_small_rowmax_fn(w, data, ref))
+                                  budgets=budgets, score_fn=_small_rowmax_fn(w, data, ref))
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # outputs on query rows whose lists match the oracle exactly
     o = o.float().cpu().numpy()
@@ -221,27 +230,31 @@ def test_prefill_end_to_end(sb, name):
             if same[hs, i]:
                 mask[h, i * w.block_size:(i + 1) * w.block_size] = True
     mx, mean = PT.output_errors(o[mask], ref["o"][mask])
+    PT.record("prefill", name, rows=exact + tie, exact=exact, tie=tie,
+              sigma_band_tiles=PT.sigma_band_tiles(budgets), max_abs=mx, mean_abs=mean)
     assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
 
 
 @pytest.mark.parametrize("name", ["rowmax_small", "rowmax_msa_small"])
 def test_rowmax_tile_scores_match_oracle(sb, name):
-    """The tensor-core row-max scores against the oracle's (bf16 centroids,
-    exact products, float64 sums) for every (selection head, tile, j < i)."""
+    """The tensor-core row-max scores against the oracle's (the largest
+    exact row score over the tile's rows, from the same fp32 centroids, in
+    float64) for every (selection head, tile, j < i), within the tie band."""
     w, data, ref = small_case(name)
     p = sb.params_for(w)
     d = _dev(data)
     qs = d["q_idx"] if w.index_dim else d["q"]
-    kc = torch.tensor(ref["c"], dtype=torch.float32, device="cuda")
-    got = sb.score_rowmax(p, qs, kc).cpu().numpy()
+    c32 = np.asarray(ref["c"], dtype=np.float32)
+    got = sb.score_rowmax(p, qs, torch.tensor(c32, device="cuda")).cpu().numpy()
     assert sb.get_status() == sb.OK
-    fn = _small_rowmax_fn(w, data, ref)
+    fn = _rowmax_fn(w, data["q_idx"] if w.index_dim else data["q"], c32.astype(np.float64))
     worst = 0.0
     for hs in range(w.n_sel_heads):
         for i in range(1, w.n_blocks):
             want = fn(hs, i).astype(np.float64)
             err = np.abs(got[hs, i, :i] - want) / np.maximum(1.0, np.abs(want))
             worst = max(worst, float(err.max()))
+    PT.record("rowmax_scores", name, worst_rel_err=worst, band=PT.BAND)
     assert worst <= PT.BAND, worst
 
 
@@ -314,9 +327,9 @@ def test_full_size_sampled(sb, name):
     gc_full = np.zeros((w.n_sel_heads, nb), dtype=np.int32)
     gi_full[:, blocks] = gidx
     gc_full[:, blocks] = gcnt
+    budgets = _budgets(w, info)
     exact, tie = PT.compare_lists(gi_full, gc_full, idx, cnt, sel_rows, qbar, c, r, w,
-                                  _kv_of_sel(w), minmax=mmx, budgets=_budgets(w, info),
-                                  score_fn=rfn)
+                                  _kv_of_sel(w), minmax=mmx, budgets=budgets, score_fn=rfn)
     assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
     # outputs of the sampled blocks whose lists match (all query heads; two
     # per group for the 64-head workload); keys/values converted once per
@@ -341,6 +354,8 @@ def test_full_size_sampled(sb, name):
     assert errs
     mx = max(e[0] for e in errs)
     mean = float(np.mean([e[1] for e in errs]))
+    PT.record("full_size_sampled", name, rows=exact + tie, exact=exact, tie=tie,
+              sigma_band_tiles=PT.sigma_band_tiles(budgets), max_abs=mx, mean_abs=mean)
     assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
 
 

@@ -119,3 +119,32 @@ def test_two_ranks_split_one_sequence_by_kv_head():
     import bench
     # one sequence of 131072 tokens, 3 steps, slowest rank 30 ms
     assert bench.weak_throughput(131072, 1, 3, 30.0) == pytest.approx(131072 * 3 / 0.03)
+
+
+# ------------------------------------------------ self-launching ranks
+
+def _bench(*args, timeout=240):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], cwd=root, env=env,
+                       capture_output=True, text=True, timeout=timeout)
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return r.returncode, (json.loads(lines[-1]) if lines else None), r.stderr
+
+
+def test_gpus_two_starts_two_ranks_itself():
+    """`bench.py --gpus 2` outside torchrun starts both ranks on this node (gloo
+    here, no GPU); rank 0 reports a world of two."""
+    rc, line, err = _bench("--gpus", "2", "--launch-check")
+    assert rc == 0, err
+    assert line["n_gpus"] == 2 and sorted(line["ranks"]) == [0, 1]
+
+
+def test_gpus_beyond_the_visible_devices_fails_loudly():
+    rc, line, err = _bench("--gpus", "4096", "--launch-check")
+    assert rc != 0 and line is None
+    assert "visible" in err

@@ -539,13 +539,34 @@ def test_percentile_gate_breaks_equal_margins_by_lower_tile():
 # score is the largest score among the tile's query rows)
 # --------------------------------------------------------------------------
 
-def test_bf16_rounding_is_round_to_nearest_even():
-    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -7, -2.0 - 2 ** -7],
-                 dtype=np.float32)
-    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: even (1); 1 + 3*2^-8 -> 1 + 2^-6;
-    # -2 - 2^-7 is halfway between -2 and -2 - 2^-6: even (-2)
-    assert O.bf16_round(x).tolist() == [1.0, 1.0, 1.0 + 2 ** -6, 1.0 + 2 ** -7, -2.0]
-    assert np.array_equal(O.bf16_round(x), torch.tensor(x).bfloat16().double().numpy())
+def test_rowmax_equals_exact_fraction_brute_force():
+    """Every tile score against exact rational arithmetic over the explicit
+    rows: max_t sum_d q_td * c_jd, times the scale, rounded to float32 once."""
+    from fractions import Fraction
+    rng = np.random.default_rng(40)
+    c = rng.standard_normal((5, 8)).astype(np.float32).astype(np.float64)
+    rows = rng.standard_normal((7, 8)).astype(np.float32).astype(np.float64)
+    scale = 0.125
+    got = O.block_scores_rowmax(rows, c, 5, scale)
+    for j in range(5):
+        best = max(sum(Fraction(float(q[d])) * Fraction(float(c[j, d])) for d in range(8))
+                   for q in rows)
+        assert got[j] == np.float32(float(best * Fraction(scale))), j
+
+
+def test_rowmax_ranks_by_the_centroids_as_given_not_rounded_to_bf16():
+    """Two candidates whose order flips if the centroids were rounded to
+    bfloat16 first: c0 = (1 + 2^-9, 0) would round to (1, 0), and c1 =
+    (1, 2^-10) is exact in bfloat16.  Against the row q = (1, 1) the exact
+    scores are 1 + 2^-9 > 1 + 2^-10, so c0 ranks first; rounded operands
+    would put c1 first."""
+    c = np.array([[1.0 + 2 ** -9, 0.0], [1.0, 2 ** -10]])
+    rows = np.array([[1.0, 1.0], [0.0, -1.0]])
+    s = O.block_scores_rowmax(rows, c, 2, 1.0).astype(np.float64)
+    assert s.tolist() == [1.0 + 2 ** -9, 1.0 + 2 ** -10]
+    assert O.top_k(s, 1).tolist() == [0]
+    rounded = torch.tensor(c, dtype=torch.float32).bfloat16().double().numpy()
+    assert (rounded @ rows[0]).tolist() == [1.0, 1.0 + 2 ** -10]   # the flip it avoids
 
 
 def test_rowmax_of_identical_rows_is_the_pooled_score_and_dominates_it_otherwise():
@@ -554,11 +575,10 @@ def test_rowmax_of_identical_rows_is_the_pooled_score_and_dominates_it_otherwise
     row = rng.standard_normal(16)
     same = np.tile(row, (32, 1))
     got = O.block_scores_rowmax(same, c, 6, 0.25)
-    want = (O.bf16_round(c) @ row * 0.25).astype(np.float32)
-    assert np.array_equal(got, want)
+    assert np.array_equal(got, O.block_scores(row, c, 6, 0.25))
     rows = rng.standard_normal((32, 16))
     mx = O.block_scores_rowmax(rows, c, 6, 0.25).astype(np.float64)
-    mean = O.bf16_round(c) @ rows.mean(axis=0) * 0.25
+    mean = c @ rows.mean(axis=0) * 0.25
     assert (mx >= mean - 1e-6).all()
     # the order of the rows does not matter
     assert np.array_equal(O.block_scores_rowmax(rows[::-1], c, 6, 0.25), mx.astype(np.float32))

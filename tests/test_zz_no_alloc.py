@@ -8,7 +8,9 @@ is fixed at start-up.  Its temporaries live in a fixed array inside the
 library instead of a caller-supplied workspace.
 
 Each case calls it through the C ABI twice in a row and checks every result
-against the workspace entry point sbsa_prefill on the same inputs.  This file
+against the workspace entry point sbsa_prefill on the same inputs, and that
+a call (after the first one on the device, which looks up the array's
+address) leaves the device's allocated and free memory unchanged.  This file
 is collected last on purpose, and passes on its own in a fresh process too.
 """
 import ctypes
@@ -78,6 +80,25 @@ def test_noalloc_matches_the_workspace_entry_point_twice(sb, name):
         assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
 
 
+def test_noalloc_allocates_no_device_memory(sb):
+    w = W.SMALL["gqa_small"]
+    data = W.generate(w, "cpu")
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in data.items()}
+    p = sb.params_for(w)
+    o = torch.empty_like(d["q"])
+    assert _noalloc(sb, p, d, o) == sb.OK            # the one-time address lookup
+    torch.cuda.synchronize()
+    before = (torch.cuda.memory_allocated(), torch.cuda.memory_reserved(),
+              torch.cuda.mem_get_info()[0])
+    for _ in range(2):
+        assert _noalloc(sb, p, d, o) == sb.OK
+    torch.cuda.synchronize()
+    after = (torch.cuda.memory_allocated(), torch.cuda.memory_reserved(),
+             torch.cuda.mem_get_info()[0])
+    assert after == before
+    assert sb.get_status() == sb.OK
+
+
 def test_noalloc_rejects_problems_larger_than_its_scratch(sb):
     # 128k tokens with the lists in the scratch: ~150 MB of temporaries
     p = sb.params_for(W.CONFIGS["rbs128k"])
@@ -90,3 +111,6 @@ def test_noalloc_rejects_problems_larger_than_its_scratch(sb):
                          block_size=128, top_k=8)
     assert fn(ctypes.byref(big), FAKE, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, None, None) == \
         sb.ERR_WORKSPACE
+    # an argument error wins over the size check, as in sbsa_prefill
+    assert fn(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, FAKE, None, FAKE, None, None) == \
+        sb.ERR_INVALID_ARG
