@@ -6,7 +6,9 @@ mass 0.9 united with the radius rescue branch).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sbsa|reference]
 
-One process per GPU (torchrun for N > 1).  By default every rank runs its
+One process per GPU.  With --gpus N > 1 and no torchrun environment the
+script starts the N ranks itself (torch.distributed.run on this node) and
+refuses N above the visible device count.  By default every rank runs its
 own independent sequence (weak scaling); with --shard heads the ranks split
 one sequence by kv head, each prefilling its kv heads and their query heads
 (strong scaling).  Neither mode has a collective on the data path: the
@@ -37,8 +39,10 @@ METRIC = "sparse prefill tokens/s and attended TFLOP/s at 128k; % of bf16 TC / H
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention launch, from the
-# ncu capture summarised in profiles/ (None until captured for this kernel).
-NCU_ATTEND_TRAFFIC = {"rbs128k": 5.608e9 + 1.050e9}
+# ncu capture summarised in profiles/, keyed by workload and by the hash of the
+# kernel source it was taken on: once that source changes the figure no longer
+# describes the kernel and the line reports null.
+NCU_ATTEND_TRAFFIC = {}
 
 
 def selection_stats(w, p, st, meta) -> dict:
@@ -78,6 +82,47 @@ def selection_stats(w, p, st, meta) -> dict:
     return out
 
 
+def source_hash(rel: str) -> str:
+    import hashlib
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def attend_kernel_source(w) -> str:
+    """The source file of the attention kernel that workload w dispatches to."""
+    name = attend_kernel_name(w)
+    base = "block_sparse_attention_sbsa_b200/csrc/"
+    for key, f in (("attend_pair", "attend_pair.cu"), ("attend_duo", "attend_duo.cu"),
+                   ("attend_ps", "attend_persist.cu")):
+        if name.startswith(key):
+            return base + f
+    return base + "attend.cu"
+
+
+def measured_traffic(w):
+    """ncu DRAM bytes of one attention launch for w, or None when none was
+    captured on the current kernel source."""
+    rec = NCU_ATTEND_TRAFFIC.get(w.name)
+    if not rec:
+        return None
+    src = attend_kernel_source(w)
+    return rec["bytes"] if rec.get("source") == src and rec.get("sha") == source_hash(src) else None
+
+
+def spread(xs):
+    """Median and 10th / 90th percentiles of per-step times (ms)."""
+    ys = sorted(xs)
+    if not ys:
+        return {}
+
+    def q(f):
+        k = f * (len(ys) - 1)
+        lo = int(math.floor(k))
+        hi = min(lo + 1, len(ys) - 1)
+        return ys[lo] + (ys[hi] - ys[lo]) * (k - lo)
+    return {"median": q(0.5), "p10": q(0.1), "p90": q(0.9), "mean": statistics.mean(ys)}
+
+
 def attend_kernel_name(w) -> str:
     """The attention kernel sbsa_attend dispatches to for workload w (the rule
     of launch_attend in csrc/attend.cu)."""
@@ -105,7 +150,7 @@ def launches_per_step(w) -> int:
     return n + 1
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
@@ -121,7 +166,9 @@ def parse_args():
                          "sequence split by kv head (strong scaling)")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override the workload length (small cases for profiling)")
-    return ap.parse_args()
+    ap.add_argument("--launch-check", action="store_true",
+                    help="only start the ranks, join the process group and report the world")
+    return ap.parse_args(argv)
 
 
 def pick_workload(args):
@@ -210,7 +257,9 @@ class ClockSampler:
 # ---------------------------------------------------------- CPU oracle leg
 def oracle_sample(w, data_cpu, blocks):
     """Oracle work for the full key pooling plus selection and attention of
-    the given query blocks (all heads).  Returns (t_pool, t_rows) seconds."""
+    the given query blocks (all heads).  Returns the two timings and what the
+    oracle computed (lists, tables, outputs of the sampled blocks) so that the
+    GPU's results can be compared with it afterwards."""
     import numpy as np
     import oracle as O
     t0 = time.perf_counter()
@@ -222,7 +271,7 @@ def oracle_sample(w, data_cpu, blocks):
     nb, b = w.n_blocks, w.block_size
     grp = w.group if w.group_shared else 1
     qbar = np.zeros((w.n_sel_heads, nb, w.score_dim))
-    sigma_gate, fired = None, None
+    sigma_gate, fired, sbar = None, None, None
     kv_of = (lambda hs: hs) if w.group_shared else (lambda hs: hs // w.group)
     if w.gate_quantile is not None:
         # the gate's global part (every tile's margin and the tile decisions)
@@ -233,7 +282,7 @@ def oracle_sample(w, data_cpu, blocks):
         O.select(qbar, c, r, block_count=nb, mode=w.select_mode, top_k_=w.top_k,
                  scale=1.0 / math.sqrt(w.score_dim), kv_of_sel=kv_of, max_blocks=w.max_blocks,
                  rows=[], minmax=minmax, sigma_gate=sigma_gate, info=info)
-        fired = info["fired"]
+        fired, sbar = info["fired"], info["sbar"]
     t_pool = time.perf_counter() - t0
     t1 = time.perf_counter()
     qsrc = data_cpu["q_rows_idx"] if w.index_dim else data_cpu["q_rows"]
@@ -256,14 +305,18 @@ def oracle_sample(w, data_cpu, blocks):
                            max_blocks=w.max_blocks, rows=rows, minmax=minmax,
                            sigma_gate=sigma_gate, row_scores=row_scores, fired=fired)
     scale = 1.0 / math.sqrt(w.head_dim)
+    outs = {}
     for bi, i in enumerate(blocks):
         for h in range(w.n_q_heads):
             hs = h // w.group if w.group_shared else h
             ids = [int(x) for x in idx[hs, i, :cnt[hs, i]]]
-            O.attend_block(data_cpu["q_rows"][h, bi * b:(bi + 1) * b], data_cpu["k"][h // w.group],
-                           data_cpu["v"][h // w.group], ids, i, b, scale)
+            outs[(h, i)] = O.attend_block(data_cpu["q_rows"][h, bi * b:(bi + 1) * b],
+                                          data_cpu["k"][h // w.group], data_cpu["v"][h // w.group],
+                                          ids, i, b, scale)
     t_rows = time.perf_counter() - t1
-    return t_pool, t_rows
+    return dict(t_pool=t_pool, t_rows=t_rows, idx=idx, cnt=cnt, rows=rows, qbar=qbar, c=c, r=r,
+                minmax=minmax, row_scores=row_scores, fired=fired, sbar=sbar, outs=outs,
+                kv_of=kv_of)
 
 
 def cpu_copy_for_oracle(w, data, blocks):
@@ -291,6 +344,24 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+class CpuMeter:
+    """Wall and process CPU time of a region: their ratio is the number of
+    host cores the region kept busy on average."""
+
+    def __enter__(self):
+        self.w0, self.c0 = time.perf_counter(), time.process_time()
+        return self
+
+    def __exit__(self, *exc):
+        self.wall = time.perf_counter() - self.w0
+        self.cpu = time.process_time() - self.c0
+        return False
+
+    @property
+    def cores(self) -> float:
+        return round(self.cpu / self.wall, 2) if self.wall > 0 else 0.0
+
+
 def sample_blocks(w, count, salt=0):
     import torch
     g = torch.Generator().manual_seed(w.seed + 101 + salt)
@@ -300,22 +371,67 @@ def sample_blocks(w, count, salt=0):
     return sorted(picks)
 
 
-def cpu_baseline_value(w, data, nblocks):
+def parity_on_sample(w, res, gpu_idx, gpu_cnt, gpu_o, blocks):
+    """The GPU's lists and outputs of the sampled query blocks against the
+    oracle's: rows equal to the oracle's, rows that differ only inside the fp32
+    tie band, and output errors over the rows whose lists are equal."""
+    import numpy as np
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import parity as PT
+    nb = w.n_blocks
+    gi = np.full((w.n_sel_heads, nb, w.max_blocks), -1, dtype=np.int32)
+    gc = np.zeros((w.n_sel_heads, nb), dtype=np.int32)
+    gi[:, blocks] = gpu_idx[:, blocks].cpu().numpy()
+    gc[:, blocks] = gpu_cnt[:, blocks].cpu().numpy()
+    budgets = None
+    if w.gate_quantile is not None:
+        budgets = PT.percentile_budgets(res["sbar"], res["fired"], w.top_k, w.gate_rho)
+    exact, tie = PT.compare_lists(gi, gc, res["idx"], res["cnt"], res["rows"], res["qbar"],
+                                  res["c"], res["r"], w, res["kv_of"], minmax=res["minmax"],
+                                  budgets=budgets, score_fn=res["row_scores"])
+    errs = []
+    b = w.block_size
+    for (h, i), ref in res["outs"].items():
+        hs = h // w.group if w.group_shared else h
+        if not np.array_equal(gi[hs, i], res["idx"][hs, i]):
+            continue
+        got = gpu_o[h, i * b:min(w.seq_len, (i + 1) * b)].float().cpu().numpy()
+        errs.append(PT.output_errors(got, ref))
+    return {"rows": exact + tie, "exact": exact, "tie": tie,
+            "sigma_band_tiles": PT.sigma_band_tiles(budgets),
+            "max_abs": max(e[0] for e in errs) if errs else None,
+            "mean_abs": float(np.mean([e[1] for e in errs])) if errs else None,
+            "bounds": {"max_abs": PT.MAX_ABS, "mean_abs": PT.MEAN_ABS, "tie_band": PT.BAND},
+            "sample": f"{len(blocks)} query blocks x {w.n_sel_heads} selection heads "
+                      f"(outputs of all {w.n_q_heads} query heads)"}
+
+
+def cpu_baseline_and_parity(w, data, nblocks, gpu_idx, gpu_cnt, gpu_o):
     blocks = sample_blocks(w, nblocks)
     cdata = cpu_copy_for_oracle(w, data, blocks)
-    t_pool, t_rows = oracle_sample(w, cdata, blocks)
+    with CpuMeter() as m:
+        res = oracle_sample(w, cdata, blocks)
+    t_pool, t_rows = res["t_pool"], res["t_rows"]
     full = t_pool + t_rows * w.n_blocks / len(blocks)
-    return {
-        "value": w.seq_len / full, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    base = {
+        "value": w.seq_len / full, "unit": UNIT, "cores": m.cores, "kind": "oracle",
+        "threads_available": blas_threads(),
         "sample": (f"numpy float64 oracle: key pooling of all {w.n_blocks} blocks "
                    f"({t_pool:.1f}s) + selection and attention of {len(blocks)} query blocks x "
                    f"{w.n_q_heads} heads ({t_rows:.1f}s), extrapolated per query block to the "
-                   f"full {w.seq_len}-token prefill ({full:.0f}s)"),
+                   f"full {w.seq_len}-token prefill ({full:.0f}s); cores = process CPU time / "
+                   f"wall time of the sample"),
     }
+    return base, parity_on_sample(w, res, gpu_idx, gpu_cnt, gpu_o, blocks)
 
 
 # ------------------------------------------------------------ reference arm
 def run_reference(args):
+    """The oracle as it stands, on the host cores: each step is a bounded
+    sample of the workload (key pooling of all blocks, selection and
+    attention of one query block in all heads); ms_per_step is the measured
+    time of that sample and the value extrapolates it per query block to the
+    full prefill."""
     import torch
     from block_sparse_attention_sbsa_b200 import workloads as W
     rank = int(os.environ.get("RANK", "0"))
@@ -324,25 +440,33 @@ def run_reference(args):
     w = pick_workload(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     data = W.generate(w, dev)
-    total_t, total_tok = 0.0, 0
+    sample_s, full_s, cpu_s = 0.0, 0.0, 0.0
     for s in range(args.warmup + args.steps):
         blocks = sample_blocks(w, 1, salt=s)
         cdata = cpu_copy_for_oracle(w, data, blocks)
-        t_pool, t_rows = oracle_sample(w, cdata, blocks)
+        with CpuMeter() as m:
+            res = oracle_sample(w, cdata, blocks)
         if s >= args.warmup:
-            total_t += t_pool + t_rows * w.n_blocks / len(blocks)
-            total_tok += w.seq_len
-    value = total_tok / total_t
+            sample_s += m.wall
+            cpu_s += m.cpu
+            full_s += res["t_pool"] + res["t_rows"] * w.n_blocks / len(blocks)
+    value = w.seq_len * args.steps / full_s
+    cores = round(cpu_s / sample_s, 2) if sample_s > 0 else 0.0
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * total_t / max(1, args.steps), "higher_is_better": True,
+        "ms_per_step": 1000.0 * sample_s / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        "extrapolated": {"ms_per_full_prefill": 1000.0 * full_s / max(1, args.steps),
+                         "note": "value = tokens of a full prefill / the sampled step's time "
+                                 "scaled per query block; ms_per_step is the sample as timed"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "threads_available": blas_threads(),
                          "sample": ("per step: key pooling of all blocks + selection and "
                                     "attention of 1 query block x all heads, extrapolated per "
-                                    "query block to the full prefill")},
+                                    "query block to the full prefill; cores = process CPU time "
+                                    "/ wall time")},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -422,9 +546,68 @@ def weak_throughput(seq_len: int, world: int, steps: int, max_ms: float) -> floa
     return seq_len * world * steps / (max_ms / 1000.0)
 
 
+# ------------------------------------------------------------- launching
+def free_port() -> int:
+    import socket
+    so = socket.socket()
+    so.bind(("127.0.0.1", 0))
+    port = so.getsockname()[1]
+    so.close()
+    return port
+
+
+def visible_devices() -> int:
+    import torch
+    return torch.cuda.device_count()
+
+
+def relaunch(args, argv) -> int:
+    """--gpus N > 1 without a torchrun environment: start the N ranks on this
+    node (one process per GPU) and return their exit status."""
+    n = visible_devices() if not args.launch_check else (visible_devices() or os.cpu_count())
+    if args.gpus > n:
+        raise SystemExit(f"--gpus {args.gpus}: only {n} device(s) visible")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
+def launch_check(args) -> int:
+    """Each rank joins the process group (NCCL on GPUs, gloo on CPU) and
+    reports itself; rank 0 prints the world it saw."""
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    dev = "cpu"
+    if backend == "nccl":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dev = "cuda"
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group(backend, timeout=timedelta(seconds=60))
+    ranks = [rank]
+    if world > 1:
+        got = [None] * world
+        dist.all_gather_object(got, rank)
+        ranks = got
+    if rank == 0:
+        print(json.dumps({"n_gpus": world, "ranks": ranks, "backend": backend, "device": dev}))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
-def main():
-    args = parse_args()
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.impl != "reference":
+        return relaunch(args, argv)
+    if args.launch_check:
+        return launch_check(args)
     if args.impl == "reference":
         return run_reference(args)
     import torch
@@ -435,6 +618,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
     if world > 1:
         from datetime import timedelta
@@ -483,6 +668,7 @@ def main():
     pairs = sbsa.attended_pairs(p, st.cnt)
     attend_flops = 4.0 * w.head_dim * pairs
     mean_cnt = float(st.cnt.float().mean())
+    valid_entries = int(st.cnt.to(torch.int64).sum())
     # planted needles are indexed by the full problem's kv heads
     sel_stats = selection_stats(w, p, st, {} if heads else data.get("meta", {}))
 
@@ -503,9 +689,11 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
-    pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    sel_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    att_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    pool_t = [e[0].elapsed_time(e[1]) for e in evs]
+    sel_t = [e[1].elapsed_time(e[2]) for e in evs]
+    att_t = [e[2].elapsed_time(e[3]) for e in evs]
+    step_t = [e[0].elapsed_time(e[3]) for e in evs]
+    pool_ms, sel_ms, att_ms = (statistics.mean(x) for x in (pool_t, sel_t, att_t))
     stat = sbsa.get_status()
     if stat != sbsa.OK:
         raise RuntimeError(f"device status after timing: {sbsa.status_string(stat)}")
@@ -556,11 +744,14 @@ def main():
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     # algorithmic bytes of pooling + selection: read Q and K (or the index
-    # tensors) once, write the fp32 tables, read them back, write the lists
+    # tensors) once, write the fp32 tables and read them back, write the valid
+    # list entries, the counts and the flags; the -1 padding of the fixed-width
+    # lists is reported beside it
     es = q.element_size()
     nb, hs, ds = w.n_blocks, w.n_sel_heads, w.score_dim
     tables = 4 * (hs * nb * ds + w.n_kv_heads * nb * ds + (w.n_kv_heads * nb if w.rescue_tau else 0))
-    lists = hs * nb * (4 * w.max_blocks + 4 + 1)
+    lists = 4 * valid_entries + hs * nb * (4 + 1)
+    padding = 4 * (hs * nb * w.max_blocks - valid_entries)
     sel_bytes = (qs.numel() + ks.numel()) * es + 2 * tables + lists
     sel_gbs = sel_bytes / ((pool_ms + sel_ms) / 1000.0) / 1e9
     line = {
@@ -574,16 +765,21 @@ def main():
         "roofline": {
             "bound": "tensor", "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",
             "frac": att_tflops / peak_tf,
-            "traffic": NCU_ATTEND_TRAFFIC.get(w.name),
+            "traffic": measured_traffic(w),
             "kernel": attend_kernel_name(w),
-            "note": f"peak = bf16_tflops burst, of {src}; achieved = 4*d*unmasked pairs / mean launch time",
+            "note": (f"peak = bf16_tflops burst, of {src}; achieved = 4*d*unmasked pairs / mean "
+                     f"launch time (CUDA events on the launching stream); traffic = ncu "
+                     f"dram bytes of one launch on the current kernel source, else null"),
         },
         "selection_roofline": {
             "bound": "hbm", "achieved": sel_gbs, "peak": peak_bw, "unit": "GB/s",
-            "frac": sel_gbs / peak_bw, "bytes": sel_bytes,
-            "note": f"pool + select kernels; peak = hbm_gbs copy, of {src}",
+            "frac": sel_gbs / peak_bw, "bytes": sel_bytes, "list_padding_bytes": padding,
+            "note": (f"pool + select kernels; bytes count valid list entries only (the -1 "
+                     f"padding is list_padding_bytes); peak = hbm_gbs copy, of {src}"),
         },
         "stages_ms": {"pool": pool_ms, "select": sel_ms, "attend": att_ms},
+        "stages_ms_spread": {"pool": spread(pool_t), "select": spread(sel_t),
+                             "attend": spread(att_t), "step": spread(step_t)},
         "selected_blocks_per_row": mean_cnt,
         "selection_stats": sel_stats,
         "attend_bytes": {
@@ -603,7 +799,8 @@ def main():
                 "output_matches_device_run": e2e_ok},
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_value(w, data, args.cpu_blocks)
+        line["cpu_baseline"], line["parity"] = cpu_baseline_and_parity(
+            w, data, args.cpu_blocks, st.idx, st.cnt, o)
     print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()

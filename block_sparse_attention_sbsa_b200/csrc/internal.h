@@ -62,19 +62,27 @@ cudaError_t launch_gate_tiles(const double* sigma, uint8_t* fire, int n_sel_head
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 
-// Row-max tile scores: the fp32 centroids are converted to bf16 into c_bf16,
-// then scores[hs, i, j] = max over the tile's query rows (and the group's
-// heads in group mode) of q_t . c_j * scale, for j < i.
+// Row-max tile scores: the fp32 centroids are split exactly into three bf16
+// parts (c_parts), then scores[hs, i, j] = max over the tile's query rows (and
+// the group's heads in group mode) of q_t . c_j * scale, for j < i.
 struct RowmaxArgs {
-  const void* q;         // [Hq, N, ds] bf16 (Q, or Q_idx in index mode)
-  const float* c_f32;    // [Hkv, NB, ds]
-  __nv_bfloat16* c_bf16; // [Hkv, NB, ds] scratch
+  const void* q;           // [Hq, N, ds] bf16 (Q, or Q_idx in index mode)
+  const float* c_f32;      // [Hkv, NB, ds]
+  __nv_bfloat16* c_parts;  // [3, Hkv, NB, ds] scratch (hi, mid, lo planes)
   float* scores;         // [Hs, NB, NB]
   int hq, hkv, n, nb, ds, group_shared;
   float scale;
   int* status;
 };
 cudaError_t launch_rowmax(const RowmaxArgs& a, cudaStream_t stream);
+
+// Whether the row-max kernel's shared memory (a 4-stage ring of part tiles,
+// the query tile and the running maxima of NB candidates) fits one CTA.
+bool rowmax_fits(int nb, int ds);
+
+// Whether the selection kernel's shared memory holds at least two score rows
+// of NB candidates (with the radii when the rescue branch is on).
+bool select_fits(int nb, int ds, int rescue);
 
 // Centroid block scores on the tensor cores: qc and kc are split into tf32
 // hi / lo parts (scratch), then scores[hs, i, j] = qc[hs, i] . kc[hs / kv_div, j]

@@ -96,6 +96,10 @@ int validate(const sbsa_params* p, Derived* d) {
   // the percentile gate's tile means are held in one CTA's shared memory
   if (p->gate == SBSA_GATE_PERCENTILE && (size_t)o.nb * sizeof(double) > 227 * 1024)
     return SBSA_ERR_UNSUPPORTED;
+  // the selection kernel holds at least two score rows in shared memory, the
+  // row-max kernel the running maxima of a tile's candidates
+  if (!select_fits(o.nb, o.ds, p->rescue ? 1 : 0)) return SBSA_ERR_UNSUPPORTED;
+  if (p->tile_score == SBSA_TILE_ROWMAX && !rowmax_fits(o.nb, o.ds)) return SBSA_ERR_UNSUPPORTED;
   o.sm_scale = p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt((float)p->head_dim);
   o.score_scale = p->score_scale > 0.f ? p->score_scale : 1.0f / std::sqrt((float)o.ds);
   if (d) *d = o;
@@ -115,7 +119,7 @@ bool centroid_tc(const sbsa_params* p) {
 }
 
 // Scratch of a precomputed score table, placed from offset `off`: for the
-// row-max tile scores the bf16 centroids, for the tensor-core centroid
+// row-max tile scores the three bf16 parts of the centroids, for the tensor-core centroid
 // scores the tf32 hi / lo parts of the pooled queries and the centroids;
 // then the table [Hs, NB, NB].
 struct ScoreScratch {
@@ -128,7 +132,7 @@ size_t score_scratch(const sbsa_params* p, const Derived& d, size_t off, ScoreSc
   const size_t q_bytes = (size_t)d.hs * d.nb * d.ds * 4;
   const size_t c_bytes = (size_t)p->n_kv_heads * d.nb * d.ds * 4;
   o->cbf = off;
-  if (rowmax) off = round_up(off + c_bytes / 2, 256);
+  if (rowmax) off = round_up(off + 3 * (c_bytes / 2), 256);
   o->q_hi = off;
   if (tc) off = round_up(off + q_bytes, 256);
   o->q_lo = off;
@@ -375,16 +379,16 @@ int sbsa_score_centroids(const sbsa_params* p, const float* q_cent, const float*
 size_t sbsa_score_rowmax_workspace_bytes(const sbsa_params* p) {
   Derived d;
   if (validate(p, &d) != SBSA_OK || p->tile_score != SBSA_TILE_ROWMAX) return 0;
-  return round_up((size_t)p->n_kv_heads * d.nb * d.ds * 2, 256);
+  return round_up(3 * (size_t)p->n_kv_heads * d.nb * d.ds * 2, 256);
 }
 
 namespace {
 RowmaxArgs rowmax_args(const sbsa_params* p, const Derived& d, const void* q_src,
-                       const float* k_cent, void* c_bf16, float* scores) {
+                       const float* k_cent, void* c_parts, float* scores) {
   RowmaxArgs a{};
   a.q = q_src;
   a.c_f32 = k_cent;
-  a.c_bf16 = static_cast<__nv_bfloat16*>(c_bf16);
+  a.c_parts = static_cast<__nv_bfloat16*>(c_parts);
   a.scores = scores;
   a.hq = p->n_q_heads;
   a.hkv = p->n_kv_heads;

@@ -41,6 +41,8 @@ extern "C" int sbsa_prefill_noalloc(const sbsa_params* p, const void* q, const v
                                     void* o, int32_t* idx_out, int32_t* cnt_out,
                                     uint8_t* flags_out, void* stream) {
   if (!p) return SBSA_ERR_INVALID_ARG;
+  // Argument errors take precedence over the size check, as in sbsa_prefill.
+  if ((idx_out == nullptr) != (cnt_out == nullptr)) return SBSA_ERR_INVALID_ARG;
   // Worst case: the lists are kept in the scratch too.  When the caller
   // provides idx_out/cnt_out, sbsa_prefill checks the smaller need itself.
   const size_t need = sbsa_prefill_workspace_bytes(p);

@@ -711,17 +711,22 @@ __global__ void __launch_bounds__(1024) gate_tiles_kernel(const double* sigma, u
   }
 }
 
+// Shared memory of a CTA of R score rows: the R pooled queries and score
+// rows, the per-warp histograms, the kv head's radii when rescuing.
+constexpr size_t kSelectBudget = 200 * 1024;
+size_t select_smem(int rows, int nb, int ds, int rescue) {
+  const size_t stride = (size_t)((nb + 3) & ~3) * 4;
+  return kHistBytes + (rescue ? stride : 0) + (size_t)rows * (stride + (size_t)ds * 4);
+}
+
 template <int DS>
 cudaError_t launch_ds(const SelectArgs& a, cudaStream_t stream) {
   // rows per CTA: as many (up to 16) as the score rows allow in shared memory;
   // more rows per CTA means fewer reads of each centroid row from L2
-  const size_t budget = 200 * 1024;
-  const size_t row = (size_t)((a.nb + 3) & ~3) * 4 + DS * 4;
-  const size_t fixed = kHistBytes + (a.rescue ? (size_t)((a.nb + 3) & ~3) * 4 : 0);
-  if (fixed + 16 * row <= budget) return launch_rows<DS, 16>(a, stream);
-  if (fixed + 8 * row <= budget) return launch_rows<DS, 8>(a, stream);
-  if (fixed + 4 * row <= budget) return launch_rows<DS, 4>(a, stream);
-  if (fixed + 2 * row <= budget) return launch_rows<DS, 2>(a, stream);
+  if (select_smem(16, a.nb, DS, a.rescue) <= kSelectBudget) return launch_rows<DS, 16>(a, stream);
+  if (select_smem(8, a.nb, DS, a.rescue) <= kSelectBudget) return launch_rows<DS, 8>(a, stream);
+  if (select_smem(4, a.nb, DS, a.rescue) <= kSelectBudget) return launch_rows<DS, 4>(a, stream);
+  if (select_smem(2, a.nb, DS, a.rescue) <= kSelectBudget) return launch_rows<DS, 2>(a, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -737,6 +742,10 @@ cudaError_t launch_gate_tiles(const double* sigma, uint8_t* fire, int n_sel_head
     return cudaErrorInvalidValue;
   gate_tiles_kernel<<<1, 1024, smem, stream>>>(sigma, fire, n_sel_heads, nb, top_k, quantile);
   return cudaGetLastError();
+}
+
+bool select_fits(int nb, int ds, int rescue) {
+  return select_smem(2, nb, ds, rescue) <= kSelectBudget;
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {

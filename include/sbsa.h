@@ -48,7 +48,12 @@ extern "C" {
 /* ---- status codes ---- */
 #define SBSA_OK 0
 #define SBSA_ERR_INVALID_ARG 1 /* null pointer, inconsistent shape or option  */
-#define SBSA_ERR_UNSUPPORTED 2 /* valid but not built: d, B, d_idx, dtype     */
+#define SBSA_ERR_UNSUPPORTED 2 /* valid but not built: d, B, d_idx, dtype, or
+                                  NB beyond what one CTA's shared memory holds:
+                                  the selection keeps two score rows (NB <= 23424
+                                  at d_s = 128, <= 15616 with the rescue branch), the row-max
+                                  scores a tile's running maxima (NB <= 16897 at
+                                  d_s = 128), the percentile gate NB doubles   */
 #define SBSA_ERR_WORKSPACE 3   /* workspace too small or misaligned           */
 #define SBSA_ERR_CUDA 4        /* a CUDA runtime/driver call failed           */
 #define SBSA_ERR_TIMEOUT 5     /* a kernel's bounded wait expired             */
@@ -105,7 +110,8 @@ typedef struct sbsa_params {
 #define SBSA_TILE_MEAN 0   /* the pooled (mean) query of the tile: one dot per block     */
 #define SBSA_TILE_ROWMAX 1 /* the page's tile score: the largest q_t . c_j over the
                               tile's query rows (and, per GQA group, the group's heads),
-                              a tensor-core contraction; centroids enter as bf16 */
+                              a tensor-core contraction with exact products (each fp32
+                              centroid split exactly into three bf16 parts) */
 
 /* ---- gates ([UGS] Metodologia steps 3-5) ---- */
 #define SBSA_GATE_GAP 1        /* per row: gap at the cut below margin * std -> 2k   */
@@ -196,11 +202,13 @@ int sbsa_score_centroids(const sbsa_params* p, const float* q_cent, const float*
  *   q_src    device [Hq, N, ds] bf16: Q, or Q_idx when p->index_dim is set.
  *   k_cent   device fp32 [Hkv, NB, ds] key centroids (sbsa_pool_blocks).
  *   scores   device fp32 [Hs, NB, NB] out: scores[hs, i, j] for j < i is
- *            max_t (q_t . bf16(c_j)) * score_scale over the query rows t of
+ *            max_t (q_t . c_j) * score_scale over the query rows t of
  *            block i (rows t < N) of head hs, or of every head of group hs
  *            when p->group_shared; entries j >= i are not written.
  *   workspace device, 256-byte aligned, >= sbsa_score_rowmax_workspace_bytes(p)
- *            (the bf16 copy of the centroids).
+ *            (the centroids split exactly into three bf16 parts).
+ * The products are exact (bf16 rows times the exact bf16 parts of each fp32
+ * centroid); the only rounding is the tensor core's fp32 accumulation.
  * Errors as sbsa_select, plus SBSA_ERR_UNSUPPORTED when p->tile_score is not
  * SBSA_TILE_ROWMAX.
  */
