@@ -531,20 +531,23 @@ cudaError_t launch_wait_probe(uint64_t timeout_ns, int* status, cudaStream_t str
 }
 
 int launch_attend(const AttendArgs& a, cudaStream_t stream) {
-  // 0: automatic, 1: pair, 2: persistent, 3: single
+  // 0: automatic, 1: pair, 2: persistent, 3: single, 4: duo
   static const int forced = [] {
     const char* e = std::getenv("SBSA_ATTEND_KERNEL");
     if (!e) return 0;
     if (std::strcmp(e, "pair") == 0) return 1;
     if (std::strcmp(e, "persistent") == 0) return 2;
     if (std::strcmp(e, "single") == 0) return 3;
+    if (std::strcmp(e, "duo") == 0) return 4;
     return 0;
   }();
   const bool big = a.dtype == SBSA_BF16 && a.block == 128 && (a.d == 128 || a.d == 64);
   // The pair kernel pays off when the two heads' lists coincide (one list
-  // per GQA group); with per-head lists the overlap is too small.
+  // per GQA group).  The two-tile kernel (duo) is built and tested but not
+  // chosen: measured slower than the persistent kernel on per-head lists.
   const bool pairable = big && a.group_shared && (a.hq / a.hkv) % 2 == 0;
   if (forced == 3 || !big) return launch_attend_single(a, stream);
+  if (forced == 4 && !a.group_shared) return launch_attend_duo(a, stream);
   if (forced == 2 || !pairable) return launch_attend_persistent(a, stream);
   return launch_attend_pair(a, stream);
 }

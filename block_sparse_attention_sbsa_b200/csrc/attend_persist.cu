@@ -7,9 +7,9 @@
 // attention over the preselected blocks only.
 //
 // One CTA per SM walks a static list of (query head, query block) items,
-// longest lists first.  The listed key blocks of consecutive items form one
-// stream indexed by a CTA-wide block counter g, so loads and products run
-// ahead across item boundaries.  14 warps:
+// kv-head major, longest lists first within a kv head.  The listed key blocks
+// of consecutive items form one stream indexed by a CTA-wide block counter g,
+// so loads and products run ahead across item boundaries.  14 warps:
 //   warp 0     TMA producer: Q of item t into Q[t % 2]; K_j, V_j of block g
 //              into a 4-stage ring (positions 2g, 2g + 1).  A position is
 //              reused once the product that read it has completed, which the
@@ -94,22 +94,32 @@ struct Item {
   int chunk_val;   // list[chunk_base + lane] (or -1 past the end)
 };
 
-// Item number t of this CTA (static round robin over the longest-first
-// order), read by a whole warp: each lane fetches one list entry, so up to
-// 32 entries cost one memory round trip.  `valid` counts the entries inside
-// [0, i].  Every lane of the warp must call this (and item_entry) together.
+// Item number t of this CTA (static round robin), read by a whole warp:
+// each lane fetches one list entry, so up to 32 entries cost one memory round
+// trip.  `valid` counts the entries inside [0, i].  Every lane of the warp
+// must call this (and item_entry) together.
+//
+// Items are ordered kv-head major -- every item reading kv head 0, then kv
+// head 1, ... -- so that the K and V blocks the lists name (2 * N * d * 2
+// bytes per kv head) stay in L2 while their items run; within a kv head the
+// latest query blocks (longest lists) come first and the query heads of the
+// group alternate.
 __device__ __forceinline__ bool load_item(const PSParams& p, int t, Item& it, int lane) {
   const long long item = (long long)blockIdx.x + (long long)t * gridDim.x;
   if (item >= p.total) return false;
-  it.i = p.nb - 1 - (int)(item / p.hq);
-  it.h = (int)(item % p.hq);
-  it.g = it.h / p.group;
+  const long long per_g = (long long)p.group * p.nb;
+  it.g = (int)(item / per_g);
+  const int r = (int)(item % per_g);
+  it.i = p.nb - 1 - r / p.group;
+  it.h = it.g * p.group + r % p.group;
   const int hs = p.group_shared ? it.g : it.h;
   it.list = p.idx + ((size_t)hs * p.nb + it.i) * p.kmax;
+  // the count and the first 32 entries are read together (one round trip)
   const int c = p.cnt[(size_t)hs * p.nb + it.i];
+  const int e0 = lane < p.kmax ? it.list[lane] : -1;
   it.count = c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
   it.chunk_base = 0;
-  it.chunk_val = lane < it.count ? it.list[lane] : -1;
+  it.chunk_val = lane < it.count ? e0 : -1;
   int v = __popc(__ballot_sync(0xFFFFFFFFu, it.chunk_val >= 0 && it.chunk_val <= it.i));
   for (int base = 32; base < it.count; base += 32) {
     const int x = base + lane < it.count ? it.list[base + lane] : -1;

@@ -116,9 +116,9 @@ struct AttendArgs {
 // Returns an SBSA_* code (SBSA_ERR_CUDA on launch/driver failure).  bf16
 // with 128-token blocks runs the head-pair kernel for lists shared by a GQA
 // group with an even number of query heads, else the persistent kernel;
-// every other combination runs the one-tile-per-CTA kernel.  The environment variable
-// SBSA_ATTEND_KERNEL ("pair", "persistent", "single") overrides the choice
-// where the requested kernel supports the arguments.
+// every other combination runs the one-tile-per-CTA kernel.  The environment variable SBSA_ATTEND_KERNEL
+// ("duo", "pair", "persistent", "single") overrides the choice where the
+// requested kernel supports the arguments.
 int launch_attend(const AttendArgs& a, cudaStream_t stream);
 
 // The head-pair kernel (bf16, B = 128, d in {64, 128}, even group size).
@@ -129,6 +129,10 @@ int launch_attend_single(const AttendArgs& a, cudaStream_t stream);
 
 // The persistent pipelined kernel (bf16, B = 128, d in {64, 128}).
 int launch_attend_persistent(const AttendArgs& a, cudaStream_t stream);
+
+// Two independent query tiles per CTA (bf16, B = 128, d in {64, 128}, one
+// list per query head).
+int launch_attend_duo(const AttendArgs& a, cudaStream_t stream);
 
 // One CTA waiting on an mbarrier that never completes, through the bounded
 // wait of the pipelines; records SBSA_ERR_TIMEOUT when the limit expires.

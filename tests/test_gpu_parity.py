@@ -445,11 +445,11 @@ def test_bounded_wait_reports_timeout_and_context_survives(sb):
     assert mx <= PT.MAX_ABS
 
 
-@pytest.mark.parametrize("kernel", ["single", "persistent", "pair"])
+@pytest.mark.parametrize("kernel", ["single", "persistent", "pair", "duo"])
 def test_alternative_attention_kernels_match_oracle_too(sb, kernel):
     """Each attention kernel forced by SBSA_ATTEND_KERNEL (one tile per CTA,
-    persistent one-tile stream, head pairs) on the 128-token-block
-    workloads, in a child process."""
+    persistent one-tile stream, head pairs, two independent tiles) on the
+    128-token-block workloads, in a child process."""
     import os
     import subprocess
     import sys
