@@ -93,7 +93,7 @@ def attend_kernel_source(w) -> str:
     name = attend_kernel_name(w)
     base = "block_sparse_attention_sbsa_b200/csrc/"
     for key, f in (("attend_pair", "attend_pair.cu"), ("attend_duo", "attend_duo.cu"),
-                   ("attend_ps", "attend_persist.cu")):
+                   ("attend_ps64", "attend_ps64.cu"), ("attend_ps", "attend_persist.cu")):
         if name.startswith(key):
             return base + f
     return base + "attend.cu"
@@ -129,6 +129,9 @@ def attend_kernel_name(w) -> str:
     big = w.dtype == "bf16" and w.block_size == 128 and w.head_dim in (64, 128)
     pairable = big and w.group_shared and (w.n_q_heads // w.n_kv_heads) % 2 == 0
     shape = f"{w.dtype}, B={w.block_size}, d={w.head_dim}"
+    if w.dtype == "bf16" and w.block_size == 64:
+        return (f"attend_ps64_kernel<{w.head_dim}> (persistent, tiles of two 64-token query "
+                f"blocks, tcgen05, {shape})")
     if pairable:
         return f"attend_pair_kernel<{w.head_dim}> (two query heads share K/V, tcgen05, {shape})"
     if big:

@@ -20,6 +20,7 @@ LIB = os.path.join(PKG, "libsbsa.so")
 SOURCES = ["pool.cu", "select.cu", "score_rowmax.cu", "score_centroid.cu", "attend.cu",
            "attend_persist.cu",
            "attend_duo.cu",
+           "attend_ps64.cu",
            "attend_pair.cu",
            "sbsa_api.cu",
            "sbsa_noalloc.cu"]

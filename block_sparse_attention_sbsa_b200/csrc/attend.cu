@@ -541,6 +541,9 @@ int launch_attend(const AttendArgs& a, cudaStream_t stream) {
     if (std::strcmp(e, "duo") == 0) return 4;
     return 0;
   }();
+  // bf16 with 64-token blocks: the persistent kernel on two-block tiles
+  if (a.dtype == SBSA_BF16 && a.block == 64 && forced != 3 && forced != 4)
+    return launch_attend_persistent64(a, stream);
   const bool big = a.dtype == SBSA_BF16 && a.block == 128 && (a.d == 128 || a.d == 64);
   // The pair kernel pays off when the two heads' lists coincide (one list
   // per GQA group).  The two-tile kernel (duo) is built and tested but not

@@ -115,8 +115,9 @@ struct AttendArgs {
 
 // Returns an SBSA_* code (SBSA_ERR_CUDA on launch/driver failure).  bf16
 // with 128-token blocks runs the head-pair kernel for lists shared by a GQA
-// group with an even number of query heads, else the persistent kernel;
-// every other combination runs the one-tile-per-CTA kernel.  The environment variable SBSA_ATTEND_KERNEL
+// group with an even number of query heads, else the persistent kernel; bf16
+// with 64-token blocks runs the persistent kernel on two-block tiles; fp32
+// runs the one-tile-per-CTA kernel.  The environment variable SBSA_ATTEND_KERNEL
 // ("duo", "pair", "persistent", "single") overrides the choice where the
 // requested kernel supports the arguments.
 int launch_attend(const AttendArgs& a, cudaStream_t stream);
@@ -129,6 +130,10 @@ int launch_attend_single(const AttendArgs& a, cudaStream_t stream);
 
 // The persistent pipelined kernel (bf16, B = 128, d in {64, 128}).
 int launch_attend_persistent(const AttendArgs& a, cudaStream_t stream);
+
+// The persistent pipelined kernel on tiles of two 64-token query blocks
+// (bf16, B = 64, d in {64, 128}).
+int launch_attend_persistent64(const AttendArgs& a, cudaStream_t stream);
 
 // Two independent query tiles per CTA (bf16, B = 128, d in {64, 128}, one
 // list per query head).

@@ -449,7 +449,8 @@ def test_bounded_wait_reports_timeout_and_context_survives(sb):
 def test_alternative_attention_kernels_match_oracle_too(sb, kernel):
     """Each attention kernel forced by SBSA_ATTEND_KERNEL (one tile per CTA,
     persistent one-tile stream, head pairs, two independent tiles) on the
-    128-token-block workloads, in a child process."""
+    128- and 64-token-block workloads, in a child process (a kernel that does
+    not take a workload's shape leaves it to the automatic choice)."""
     import os
     import subprocess
     import sys
@@ -458,7 +459,7 @@ def test_alternative_attention_kernels_match_oracle_too(sb, kernel):
         "import test_gpu_parity as T, numpy as np, torch\n"
         "from block_sparse_attention_sbsa_b200 import sbsa\n"
         "import parity as PT\n"
-        "for name in ['gqa_small', 'rbs_small', 'msa_small']:\n"
+        "for name in ['gqa_small', 'rbs_small', 'msa_small', 'gate_small', 'sigma_small']:\n"
         "    w, data, ref = T.small_case(name)\n"
         "    d = T._dev(data)\n"
         "    o = sbsa.attend(sbsa.params_for(w), d['q'], d['k'], d['v'],\n"
