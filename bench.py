@@ -42,7 +42,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # ncu capture summarised in profiles/, keyed by workload and by the hash of the
 # kernel source it was taken on: once that source changes the figure no longer
 # describes the kernel and the line reports null.
-NCU_ATTEND_TRAFFIC = {}
+NCU_ATTEND_TRAFFIC = {
+    # profiles/attend_ps_kernel_dram_rbs.md: 2.39 GB read + 1.05 GB written
+    "rbs128k": {"bytes": 3.44e9, "source": "block_sparse_attention_sbsa_b200/csrc/attend_persist.cu",
+                "sha": "69163a631d3ab4b5"},
+}
 
 
 def selection_stats(w, p, st, meta) -> dict:

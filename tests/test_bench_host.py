@@ -50,3 +50,20 @@ def test_sampler_without_the_tool_reports_nothing(tmp_path, monkeypatch):
     c = bench.ClockSampler(0)
     c.start()
     assert c.stop() is None
+
+
+def test_traffic_is_reported_only_for_the_kernel_source_it_was_taken_on(monkeypatch):
+    from block_sparse_attention_sbsa_b200 import workloads as W
+    w = W.CONFIGS["rbs128k"]
+    rec = bench.NCU_ATTEND_TRAFFIC["rbs128k"]
+    assert bench.attend_kernel_source(w) == rec["source"]
+    same = bench.source_hash(rec["source"]) == rec["sha"]
+    assert bench.measured_traffic(w) == (rec["bytes"] if same else None)
+    monkeypatch.setattr(bench, "source_hash", lambda rel: "0" * 16)
+    assert bench.measured_traffic(w) is None                   # any other source
+    assert bench.measured_traffic(W.CONFIGS["gqa32k"]) is None  # never captured
+
+
+def test_spread_reports_median_and_deciles():
+    s = bench.spread([float(x) for x in range(1, 12)])
+    assert s["median"] == 6.0 and s["p10"] == 2.0 and s["p90"] == 10.0 and s["mean"] == 6.0
