@@ -11,9 +11,11 @@ script starts the N ranks itself (torch.distributed.run on this node) and
 refuses N above the visible device count.  By default every rank runs its
 own independent sequence (weak scaling); with --shard heads the ranks split
 one sequence by kv head, each prefilling its kv heads and their query heads
-(strong scaling).  Neither mode has a collective on the data path: the
-selection and the attention of a kv head need nothing from another.  The
-reported time is the maximum over ranks.  Rank 0 prints one JSON line.
+(strong scaling).  The selection and the attention of a kv head need
+nothing from another, with one exception: the percentile gate averages a
+tile's cut margins over every head, so under --shard heads its per-tile
+margin sums are all-reduced (NCCL) between its two halves.  The reported
+time is the maximum over ranks.  Rank 0 prints one JSON line.
 `--impl reference` times the CPU oracle on a bounded sample of the same
 workload instead.
 """
@@ -145,15 +147,16 @@ def attend_kernel_name(w) -> str:
 
 def launches_per_step(w) -> int:
     """Kernels one staged prefill step launches (the calls of sbsa.Staged):
-    key pooling; query pooling, or the bf16 conversion and row-max scores;
-    with the mean backbone and mean tile scores the tf32 split and the
-    tensor-core centroid scores; the selection (three launches under the
-    percentile gate); the attention."""
+    key pooling; query pooling, or the three-part centroid split and the
+    row-max scores; with the mean backbone and mean tile scores the tf32 split
+    and the tensor-core centroid scores; the selection (four launches under
+    the percentile gate: first pass, per-tile sums, tile decisions, second
+    pass); the attention."""
     rowmax = w.tile_score == "rowmax"
     n = 1 + (2 if rowmax else 1)
     if w.backbone == "mean" and not rowmax and w.n_blocks >= 2:
         n += 2
-    n += 3 if w.gate_quantile is not None else 1
+    n += 4 if w.gate_quantile is not None else 1
     return n + 1
 
 
@@ -633,13 +636,14 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300))
 
     heads = args.shard == "heads" and world > 1
+    exchange = None
     if heads:
         # every rank draws the same sequence and keeps its kv heads
         w_full = pick_workload(args)
         if w_full.gate_quantile is not None:
-            raise SystemExit("--shard heads: the percentile gate averages its margins over all "
-                             "heads of a tile, which would need an all-reduce between its "
-                             "passes; shard by sequences instead")
+            # the percentile gate averages a tile's margins over every head:
+            # one all-reduce of the per-tile sums between its two halves
+            exchange = lambda t: dist.all_reduce(t)
         w, (g0, g1) = shard_workload(w_full, rank, world)
         data = shard_tensors(W.generate(w_full, "cuda"), w_full, g0, g1)
     else:
@@ -659,7 +663,7 @@ def main(argv=None):
         st.pool(qs, ks)
         if evs:
             evs[1].record(stream)
-        st.select()
+        st.select(exchange=exchange, total_heads=w_full.n_sel_heads)
         if evs:
             evs[2].record(stream)
         st.attend(q, k, v, o)

@@ -55,10 +55,15 @@ struct SelectArgs {
   int* status;
 };
 
-// The percentile gate's tile decisions: mean margin per tile over the Hs
-// heads, the floor(q T) smallest of the T tiles with more than k candidates.
-cudaError_t launch_gate_tiles(const double* sigma, uint8_t* fire, int n_sel_heads, int nb,
-                              int top_k, float quantile, cudaStream_t stream);
+// The percentile gate's tile decisions, in two halves so that the selection
+// heads may be spread over several processes: the sum of each tile's margins
+// over this call's Hs heads (head order), then -- once the sums cover every
+// head -- the mean over total_heads and the floor(q T) smallest of the T tiles
+// with more than k candidates.
+cudaError_t launch_gate_sums(const double* sigma, double* sums, int n_sel_heads, int nb,
+                             cudaStream_t stream);
+cudaError_t launch_gate_fire(const double* sums, uint8_t* fire, int total_heads, int nb,
+                             int top_k, float quantile, cudaStream_t stream);
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 

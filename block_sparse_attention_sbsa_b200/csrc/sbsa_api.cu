@@ -146,19 +146,26 @@ size_t score_scratch(const sbsa_params* p, const Derived& d, size_t off, ScoreSc
   return off;
 }
 
+struct GateScratch {
+  size_t sigma, sums, fire;
+};
+
 struct WsLayout {
-  size_t qc, kc, kr, idx, cnt, flags, sigma, fire, total;
+  size_t qc, kc, kr, idx, cnt, flags, total;
+  GateScratch gs;
   ScoreScratch sc;
 };
 
-// Scratch of the percentile gate: per-row margins (double) and per-tile
-// decisions, placed from offset `off`.
-size_t gate_scratch(const sbsa_params* p, const Derived& d, size_t off, size_t* sigma,
-                    size_t* fire) {
-  *sigma = off;
-  if (p->gate == SBSA_GATE_PERCENTILE) off = round_up(off + (size_t)d.hs * d.nb * 8, 256);
-  *fire = off;
-  if (p->gate == SBSA_GATE_PERCENTILE) off = round_up(off + (size_t)d.nb, 256);
+// Scratch of the percentile gate, placed from offset `off`: per-row margins
+// (double), per-tile margin sums (double) and per-tile decisions.
+size_t gate_scratch(const sbsa_params* p, const Derived& d, size_t off, GateScratch* g) {
+  const bool on = p->gate == SBSA_GATE_PERCENTILE;
+  g->sigma = off;
+  if (on) off = round_up(off + (size_t)d.hs * d.nb * 8, 256);
+  g->sums = off;
+  if (on) off = round_up(off + (size_t)d.nb * 8, 256);
+  g->fire = off;
+  if (on) off = round_up(off + (size_t)d.nb, 256);
   return off;
 }
 
@@ -178,7 +185,7 @@ WsLayout layout(const sbsa_params* p, const Derived& d, bool lists) {
   off = round_up(off + (lists ? (size_t)d.hs * d.nb * 4 : 0), 256);
   w.flags = off;
   off = round_up(off + (lists ? (size_t)d.hs * d.nb : 0), 256);
-  off = gate_scratch(p, d, off, &w.sigma, &w.fire);
+  off = gate_scratch(p, d, off, &w.gs);
   off = score_scratch(p, d, off, &w.sc);
   w.total = off;
   return w;
@@ -235,22 +242,42 @@ CentroidScoreArgs centroid_args(const sbsa_params* p, const Derived& d, const fl
   return a;
 }
 
-// The selection on a stream: one launch, or for the percentile gate the
-// three of it (top-k lists and margins, tile decisions, fired tiles again).
-int run_select(const sbsa_params* p, const Derived& d, SelectArgs a, unsigned char* scratch,
-               size_t sigma_off, size_t fire_off, cudaStream_t s) {
-  if (p->gate != SBSA_GATE_PERCENTILE) return cuda_code(launch_select(a, s));
-  double* sigma = reinterpret_cast<double*>(scratch + sigma_off);
-  uint8_t* fire = scratch + fire_off;
-  a.sigma = sigma;
-  a.fire = fire;
+// The percentile gate's first pass: top-k lists and per-row margins, then
+// the per-tile sums of the margins over this call's heads into `sums`.
+int gate_first(const Derived& d, SelectArgs a, unsigned char* scratch, const GateScratch& g,
+               double* sums, cudaStream_t s) {
+  a.sigma = reinterpret_cast<double*>(scratch + g.sigma);
+  a.fire = scratch + g.fire;
   a.pass = 1;
   int rc = cuda_code(launch_select(a, s));
   if (rc) return rc;
-  rc = cuda_code(launch_gate_tiles(sigma, fire, d.hs, d.nb, p->top_k, p->gate_quantile, s));
+  return cuda_code(launch_gate_sums(a.sigma, sums, d.hs, d.nb, s));
+}
+
+// Its second pass: the tile decisions from sums that cover `total_heads`
+// heads, then top rho*k in the rows of the fired tiles.
+int gate_second(const sbsa_params* p, const Derived& d, SelectArgs a, unsigned char* scratch,
+                const GateScratch& g, const double* sums, int total_heads, cudaStream_t s) {
+  uint8_t* fire = scratch + g.fire;
+  a.sigma = reinterpret_cast<double*>(scratch + g.sigma);
+  a.fire = fire;
+  int rc = cuda_code(
+      launch_gate_fire(sums, fire, total_heads, d.nb, p->top_k, p->gate_quantile, s));
   if (rc) return rc;
   a.pass = 2;
   return cuda_code(launch_select(a, s));
+}
+
+// The selection on a stream: one launch, or for the percentile gate its
+// four (top-k lists and margins, per-tile sums, tile decisions, fired tiles
+// again).
+int run_select(const sbsa_params* p, const Derived& d, SelectArgs a, unsigned char* scratch,
+               const GateScratch& g, cudaStream_t s) {
+  if (p->gate != SBSA_GATE_PERCENTILE) return cuda_code(launch_select(a, s));
+  double* sums = reinterpret_cast<double*>(scratch + g.sums);
+  int rc = gate_first(d, a, scratch, g, sums, s);
+  if (rc) return rc;
+  return gate_second(p, d, a, scratch, g, sums, d.hs, s);
 }
 
 AttendArgs attend_args(const sbsa_params* p, const Derived& d, const void* q, const void* k,
@@ -344,9 +371,9 @@ int sbsa_select(const sbsa_params* p, const float* q_cent, const float* k_cent,
 size_t sbsa_select_workspace_bytes(const sbsa_params* p) {
   Derived d;
   if (validate(p, &d) != SBSA_OK) return 0;
-  size_t sigma, fire;
+  GateScratch g;
   ScoreScratch sc;
-  const size_t off = gate_scratch(p, d, 0, &sigma, &fire);
+  const size_t off = gate_scratch(p, d, 0, &g);
   return centroid_tc(p) ? score_scratch(p, d, off, &sc) : off;
 }
 
@@ -424,45 +451,106 @@ int sbsa_select_scores(const sbsa_params* p, const float* scores, int32_t* idx, 
   if (rc) return rc;
   if (!scores || !idx || !cnt) return SBSA_ERR_INVALID_ARG;
   if (p->rescue) return SBSA_ERR_INVALID_ARG;  // the rescue bound needs the tables
-  size_t sigma, fire;
-  const size_t need = gate_scratch(p, d, 0, &sigma, &fire);
+  GateScratch g;
+  const size_t need = gate_scratch(p, d, 0, &g);
   if (need && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
                ws_bytes < need))
     return SBSA_ERR_WORKSPACE;
   SelectArgs a = select_args(p, d, nullptr, nullptr, nullptr, idx, cnt, flags);
   a.scores = scores;
-  return run_select(p, d, a, static_cast<unsigned char*>(workspace), sigma, fire,
+  return run_select(p, d, a, static_cast<unsigned char*>(workspace), g,
                     static_cast<cudaStream_t>(stream));
 }
+
+namespace {
+// Checks and scores shared by sbsa_select_ws and the two halves of the
+// percentile gate: validates the arguments and the workspace, takes the
+// tensor-core centroid scores into it where they apply, and returns the
+// selection's arguments (rc != SBSA_OK: nothing was launched).
+struct SelectWs {
+  int rc;
+  Derived d;
+  GateScratch g;
+  SelectArgs a;
+};
+
+SelectWs select_ws_prepare(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                           const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
+                           void* workspace, size_t ws_bytes, bool scores_now,
+                           cudaStream_t s) {
+  SelectWs r{};
+  r.rc = validate(p, &r.d);
+  if (r.rc) return r;
+  const Derived& d = r.d;
+  r.rc = SBSA_ERR_INVALID_ARG;
+  if (!q_cent || !k_cent || !idx || !cnt) return r;
+  if (p->rescue && !k_radius) return r;
+  if (!aligned16(q_cent) || !aligned16(k_cent)) return r;
+  // workspace: the percentile gate's scratch, then the score table's
+  ScoreScratch sc;
+  const size_t gate_end = gate_scratch(p, d, 0, &r.g);
+  const size_t need = centroid_tc(p) ? score_scratch(p, d, gate_end, &sc) : gate_end;
+  r.rc = SBSA_ERR_WORKSPACE;
+  if (need && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+               ws_bytes < need))
+    return r;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  r.a = select_args(p, d, q_cent, k_cent, p->rescue ? k_radius : nullptr, idx, cnt, flags);
+  r.rc = SBSA_OK;
+  if (centroid_tc(p)) {
+    float* scores = reinterpret_cast<float*>(ws + sc.scores);
+    if (scores_now)
+      r.rc = cuda_code(launch_centroid_scores(centroid_args(p, d, q_cent, k_cent, ws, sc, scores), s));
+    r.a.scores = scores;  // the pooled queries stay for the rescue bound
+  }
+  return r;
+}
+}  // namespace
 
 int sbsa_select_ws(const sbsa_params* p, const float* q_cent, const float* k_cent,
                    const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
                    void* workspace, size_t ws_bytes, void* stream) {
-  Derived d;
-  int rc = validate(p, &d);
-  if (rc) return rc;
-  if (!q_cent || !k_cent || !idx || !cnt) return SBSA_ERR_INVALID_ARG;
-  if (p->rescue && !k_radius) return SBSA_ERR_INVALID_ARG;
-  if (!aligned16(q_cent) || !aligned16(k_cent)) return SBSA_ERR_INVALID_ARG;
-  // workspace: the percentile gate's scratch, then the score table's
-  size_t sigma, fire;
-  ScoreScratch sc;
-  const size_t gate_end = gate_scratch(p, d, 0, &sigma, &fire);
-  const size_t need = centroid_tc(p) ? score_scratch(p, d, gate_end, &sc) : gate_end;
-  if (need && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-               ws_bytes < need))
-    return SBSA_ERR_WORKSPACE;
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  SelectArgs a = select_args(p, d, q_cent, k_cent, p->rescue ? k_radius : nullptr, idx, cnt,
-                             flags);
-  if (centroid_tc(p)) {
-    float* scores = reinterpret_cast<float*>(ws + sc.scores);
-    rc = cuda_code(launch_centroid_scores(centroid_args(p, d, q_cent, k_cent, ws, sc, scores), s));
-    if (rc) return rc;
-    a.scores = scores;  // the pooled queries stay for the rescue bound
-  }
-  return run_select(p, d, a, ws, sigma, fire, s);
+  SelectWs r = select_ws_prepare(p, q_cent, k_cent, k_radius, idx, cnt, flags, workspace,
+                                 ws_bytes, true, s);
+  if (r.rc) return r.rc;
+  return run_select(p, r.d, r.a, static_cast<unsigned char*>(workspace), r.g, s);
+}
+
+int sbsa_select_gate_partial(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                             const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
+                             void* workspace, size_t ws_bytes, double* tile_sums,
+                             void* stream) {
+  const int rc = validate(p, nullptr);
+  if (rc) return rc;
+  if (p->gate != SBSA_GATE_PERCENTILE || p->tile_score != SBSA_TILE_MEAN)
+    return SBSA_ERR_INVALID_ARG;
+  if (!tile_sums || (reinterpret_cast<uintptr_t>(tile_sums) & 7u) != 0)
+    return SBSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SelectWs r = select_ws_prepare(p, q_cent, k_cent, k_radius, idx, cnt, flags, workspace,
+                                 ws_bytes, true, s);
+  if (r.rc) return r.rc;
+  return gate_first(r.d, r.a, static_cast<unsigned char*>(workspace), r.g, tile_sums, s);
+}
+
+int sbsa_select_gate_finish(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                            const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
+                            void* workspace, size_t ws_bytes, const double* tile_sums,
+                            int total_heads, void* stream) {
+  const int rc = validate(p, nullptr);
+  if (rc) return rc;
+  if (p->gate != SBSA_GATE_PERCENTILE || p->tile_score != SBSA_TILE_MEAN)
+    return SBSA_ERR_INVALID_ARG;
+  if (!tile_sums || (reinterpret_cast<uintptr_t>(tile_sums) & 7u) != 0)
+    return SBSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SelectWs r = select_ws_prepare(p, q_cent, k_cent, k_radius, idx, cnt, flags, workspace,
+                                 ws_bytes, false, s);
+  if (r.rc) return r.rc;
+  if (total_heads < r.d.hs) return SBSA_ERR_INVALID_ARG;
+  return gate_second(p, r.d, r.a, static_cast<unsigned char*>(workspace), r.g, tile_sums,
+                     total_heads, s);
 }
 
 int sbsa_attend(const sbsa_params* p, const void* q, const void* k, const void* v,
@@ -534,7 +622,7 @@ int sbsa_prefill(const sbsa_params* p, const void* q, const void* k, const void*
     if (rc) return rc;
     sa.scores = scores;  // the pooled queries stay for the rescue bound
   }
-  rc = run_select(p, d, sa, ws, w.sigma, w.fire, s);
+  rc = run_select(p, d, sa, ws, w.gs, s);
   if (rc) return rc;
   return launch_attend(attend_args(p, d, q, k, v, idx, cnt, o), s);
 }

@@ -680,19 +680,27 @@ cudaError_t launch_rows(const SelectArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// Percentile gate, tile decisions: the mean cut margin of each query tile
-// over the selection heads (summed in head order, double), then the
-// floor(q T) smallest of the T tiles with more than k candidates fire, lower
-// tile first on equal means.  One CTA; the means live in shared memory.
-__global__ void __launch_bounds__(1024) gate_tiles_kernel(const double* sigma, uint8_t* fire,
-                                                          int n_sel_heads, int nb, int top_k,
-                                                          float quantile) {
-  extern __shared__ double sbar[];
-  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+// Percentile gate, first half of the tile decisions: the sum of each query
+// tile's cut margins over this call's selection heads, in head order
+// (double).  Tiles with at most k candidates have no margin (NaN).
+__global__ void __launch_bounds__(256) gate_sums_kernel(const double* sigma, double* sums,
+                                                        int n_sel_heads, int nb) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nb; i += gridDim.x * blockDim.x) {
     double tot = 0.0;
     for (int h = 0; h < n_sel_heads; ++h) tot += sigma[(size_t)h * nb + i];
-    sbar[i] = tot / (double)n_sel_heads;
+    sums[i] = tot;
   }
+}
+
+// Percentile gate, second half: the mean margin of each tile is its sum over
+// all selection heads divided by their number; the floor(q T) smallest of the
+// T tiles with more than k candidates fire, lower tile first on equal means.
+// One CTA; the means live in shared memory.
+__global__ void __launch_bounds__(1024) gate_fire_kernel(const double* sums, uint8_t* fire,
+                                                         int total_heads, int nb, int top_k,
+                                                         float quantile) {
+  extern __shared__ double sbar[];
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) sbar[i] = sums[i] / (double)total_heads;
   __syncthreads();
   const int t_eligible = nb - 1 - top_k > 0 ? nb - 1 - top_k : 0;
   const int n_fire = (int)floor((double)quantile * (double)t_eligible);
@@ -732,15 +740,22 @@ cudaError_t launch_ds(const SelectArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_gate_tiles(const double* sigma, uint8_t* fire, int n_sel_heads, int nb,
-                              int top_k, float quantile, cudaStream_t stream) {
+cudaError_t launch_gate_sums(const double* sigma, double* sums, int n_sel_heads, int nb,
+                             cudaStream_t stream) {
+  const int blocks = (nb + 255) / 256;
+  gate_sums_kernel<<<blocks, 256, 0, stream>>>(sigma, sums, n_sel_heads, nb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_fire(const double* sums, uint8_t* fire, int total_heads, int nb,
+                             int top_k, float quantile, cudaStream_t stream) {
   const size_t smem = (size_t)nb * sizeof(double);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(gate_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(gate_fire_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return cudaErrorInvalidValue;
-  gate_tiles_kernel<<<1, 1024, smem, stream>>>(sigma, fire, n_sel_heads, nb, top_k, quantile);
+  gate_fire_kernel<<<1, 1024, smem, stream>>>(sums, fire, total_heads, nb, top_k, quantile);
   return cudaGetLastError();
 }
 

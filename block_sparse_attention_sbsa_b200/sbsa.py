@@ -30,7 +30,8 @@ SYMBOLS = ["sbsa_pool_blocks", "sbsa_pool_minmax", "sbsa_select", "sbsa_select_w
            "sbsa_select_workspace_bytes", "sbsa_score_centroids",
            "sbsa_score_centroids_workspace_bytes", "sbsa_score_rowmax",
            "sbsa_score_rowmax_workspace_bytes",
-           "sbsa_select_scores", "sbsa_attend", "sbsa_prefill",
+           "sbsa_select_scores", "sbsa_select_gate_partial", "sbsa_select_gate_finish",
+           "sbsa_attend", "sbsa_prefill",
            "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string",
            "sbsa_version", "sbsa_debug_wait_timeout"]
 
@@ -102,6 +103,10 @@ def _load() -> ctypes.CDLL:
     lib.sbsa_score_rowmax_workspace_bytes.argtypes = [P]
     lib.sbsa_score_rowmax_workspace_bytes.restype = ctypes.c_size_t
     lib.sbsa_select_scores.argtypes = [P, f32p, i32p, i32p, u8p, vp, ctypes.c_size_t, vp]
+    lib.sbsa_select_gate_partial.argtypes = [P, f32p, f32p, f32p, i32p, i32p, u8p, vp,
+                                             ctypes.c_size_t, vp, vp]
+    lib.sbsa_select_gate_finish.argtypes = [P, f32p, f32p, f32p, i32p, i32p, u8p, vp,
+                                            ctypes.c_size_t, vp, ci, vp]
     lib.sbsa_attend.argtypes = [P, vp, vp, vp, i32p, i32p, vp, vp]
     lib.sbsa_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i32p, i32p, u8p, vp]
     lib.sbsa_prefill_workspace_bytes.argtypes = [P]
@@ -417,6 +422,7 @@ class Staged:
         self.ws_bytes = int(lib.sbsa_select_workspace_bytes(ctypes.byref(p)))
         self.ws = (torch.empty(self.ws_bytes, device=device, dtype=torch.uint8)
                    if self.ws_bytes else None)
+        self.tile_sums = None
         self._p = ctypes.byref(p)
 
     def pool(self, q_src, k_src, stream=None):
@@ -437,7 +443,27 @@ class Staged:
         _check(lib.sbsa_pool_blocks(self._p, _ptr(q_src), p.n_q_heads, ds, grp, _ptr(self.qc),
                                     None, s), "sbsa_pool_blocks")
 
-    def select(self, stream=None):
+    def select(self, stream=None, exchange=None, total_heads=None):
+        """The selection stage.  Under the percentile gate with several
+        processes sharing one sequence by kv head, `exchange(tile_sums)` sums
+        the per-tile margin sums (a device float64 tensor [NB]) over the
+        processes in place (an all-reduce), and `total_heads` is the number of
+        selection heads over all of them; the gate then decides every tile on
+        the mean over all heads."""
+        p = self.p
+        if exchange is not None and p.gate == GATE_PERCENTILE and not self.rowmax:
+            if self.tile_sums is None:
+                self.tile_sums = torch.empty(p.n_blocks, device=self.qc.device,
+                                             dtype=torch.float64)
+            args = (self._p, _ptr(self.qc), _ptr(self.kc), _ptr(self.kr), _ptr(self.idx),
+                    _ptr(self.cnt), _ptr(self.flags), _ptr(self.ws), self.ws_bytes)
+            _check(lib.sbsa_select_gate_partial(*args, _ptr(self.tile_sums), _stream(stream)),
+                   "sbsa_select_gate_partial")
+            exchange(self.tile_sums)
+            _check(lib.sbsa_select_gate_finish(*args, _ptr(self.tile_sums),
+                                               int(total_heads or p.n_sel_heads),
+                                               _stream(stream)), "sbsa_select_gate_finish")
+            return
         if self.rowmax:
             _check(lib.sbsa_select_scores(self._p, _ptr(self.scores), _ptr(self.idx),
                                           _ptr(self.cnt), _ptr(self.flags), _ptr(self.ws),

@@ -252,6 +252,38 @@ int sbsa_select_ws(const sbsa_params* p, const float* q_cent, const float* k_cen
                    void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * sbsa_select_gate_partial / sbsa_select_gate_finish -- sbsa_select_ws under
+ * the percentile gate ([UGS] Metodologia steps 3-5), split in two so that the
+ * selection heads may be spread over several processes (one sequence sharded
+ * by kv head).  The gate is the only rule that couples heads: a tile's
+ * decision uses the mean of its cut margins over ALL selection heads.  The
+ * pages have no entry point for this; the split is this library's.
+ *   partial: centroid scores (tensor cores) into the workspace, top-k lists and
+ *            per-row margins of this call's heads, then
+ *            tile_sums[i] = sum over this call's heads (head order, double) of
+ *            the margin of tile i (NaN for tiles with at most k candidates).
+ *   The caller sums tile_sums over the processes (an all-reduce), then
+ *   finish:  mean margin = tile_sums / total_heads, the floor(q T) smallest of
+ *            the T tiles with more than k candidates fire, and the rows of the
+ *            fired tiles are redone with top rho*k.
+ *   Both calls take the same arguments as sbsa_select_ws and the SAME
+ *   workspace (finish reads the scores and margins partial left in it).
+ *   tile_sums    device double [NB], 8-byte aligned.
+ *   total_heads  selection heads over all processes (>= this call's Hs).
+ * With total_heads = Hs and tile_sums untouched between the calls the result
+ * is that of sbsa_select_ws.  Errors as sbsa_select_ws; SBSA_ERR_INVALID_ARG
+ * unless p->gate is SBSA_GATE_PERCENTILE with mean tile scores, for a missing
+ * or misaligned tile_sums, or total_heads < Hs.
+ */
+int sbsa_select_gate_partial(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                             const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
+                             void* workspace, size_t ws_bytes, double* tile_sums, void* stream);
+int sbsa_select_gate_finish(const sbsa_params* p, const float* q_cent, const float* k_cent,
+                            const float* k_radius, int32_t* idx, int32_t* cnt, uint8_t* flags,
+                            void* workspace, size_t ws_bytes, const double* tile_sums,
+                            int total_heads, void* stream);
+
+/*
  * sbsa_attend -- [RBS] sparse prefill attention; [MSA] main branch.
  *   q [Hq,N,d], k/v [Hkv,N,d], o [Hq,N,d]: device, element type p->dtype.
  *   idx/cnt: lists as produced by sbsa_select (Hs rows per p->group_shared).

@@ -212,7 +212,8 @@ def test_percentile_gate_needs_a_workspace(sb):
     p = _valid(sb, gate_quantile=0.3, gate_rho=2, seq_len=4096)
     nb = p.n_blocks
     need = sb.lib.sbsa_select_workspace_bytes(ctypes.byref(p))
-    gate = (4 * nb * 8 + 255) // 256 * 256 + (nb + 255) // 256 * 256
+    # per-row margins, per-tile margin sums (doubles), per-tile decisions
+    gate = r256(4 * nb * 8) + r256(nb * 8) + r256(nb)
     assert need == gate + _centroid_scratch(p)
     mm = _valid(sb, gate_quantile=0.3, gate_rho=2, seq_len=4096, backbone="minmax")
     assert sb.lib.sbsa_select_workspace_bytes(ctypes.byref(mm)) == gate
@@ -225,6 +226,24 @@ def test_percentile_gate_needs_a_workspace(sb):
     # the prefill workspace grows by the gate's scratch
     plain = sb.workspace_bytes(_valid(sb, seq_len=4096, max_blocks=p.max_blocks))
     assert sb.workspace_bytes(p) == plain + gate
+
+
+def test_percentile_gate_halves_check_their_arguments(sb):
+    p = _valid(sb, gate_quantile=0.3, gate_rho=2, seq_len=4096)
+    need = sb.lib.sbsa_select_workspace_bytes(ctypes.byref(p))
+    part, fin = sb.lib.sbsa_select_gate_partial, sb.lib.sbsa_select_gate_finish
+    args = (ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, None, FAKE, need)
+    assert part(*args, None, None) == 1                              # no tile sums
+    assert part(*args, ctypes.c_void_p((1 << 20) + 4), None) == 1    # misaligned
+    assert fin(*args, FAKE, p.n_sel_heads - 1, None) == 1            # fewer heads than its own
+    short = (ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, None, FAKE, need - 1)
+    assert part(*short, FAKE, None) == 3 and fin(*short, FAKE, 8, None) == 3
+    plain = _valid(sb)                                               # no percentile gate
+    assert part(ctypes.byref(plain), FAKE, FAKE, None, FAKE, FAKE, None, FAKE, 1 << 20, FAKE,
+                None) == 1
+    rowmax = _valid(sb, gate_quantile=0.3, gate_rho=2, tile_score="rowmax")
+    assert fin(ctypes.byref(rowmax), FAKE, FAKE, None, FAKE, FAKE, None, FAKE, 1 << 30, FAKE, 8,
+               None) == 1
 
 
 def test_rowmax_workspace_and_checks(sb):

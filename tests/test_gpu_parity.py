@@ -258,6 +258,60 @@ def test_rowmax_tile_scores_match_oracle(sb, name):
     assert worst <= PT.BAND, worst
 
 
+@pytest.mark.parametrize("name", ["sigma_small", "sigma_quest_small"])
+def test_percentile_gate_over_two_head_shards(sb, name):
+    """The two halves of the percentile gate (sbsa_select_gate_partial /
+    _finish) on two kv-head shards of one sequence, their per-tile margin sums
+    added on the device in between (what an all-reduce over two ranks does),
+    against the oracle's unsharded selection: the same tie-band check as the
+    single-call path."""
+    import ctypes
+    import bench
+    w, data, ref = small_case(name)
+    qc = torch.tensor(ref["qbar"], dtype=torch.float32, device="cuda")
+    if w.backbone == "minmax":
+        kc = torch.tensor(np.stack(ref["minmax"], axis=2), dtype=torch.float32, device="cuda")
+    else:
+        kc = torch.tensor(ref["c"], dtype=torch.float32, device="cuda")
+    nb = w.n_blocks
+    sums = torch.zeros(nb, dtype=torch.float64, device="cuda")
+    shards = []
+    for rank in range(2):
+        wsh, (g0, g1) = bench.shard_workload(w, rank, 2)
+        ps = sb.params_for(wsh)
+        hs0, hs1 = g0 * w.group, g1 * w.group
+        st = dict(p=ps, qc=qc[hs0:hs1].contiguous(), kc=kc[g0:g1].contiguous(),
+                  idx=torch.empty(hs1 - hs0, nb, ps.max_blocks, dtype=torch.int32, device="cuda"),
+                  cnt=torch.empty(hs1 - hs0, nb, dtype=torch.int32, device="cuda"),
+                  flags=torch.empty(hs1 - hs0, nb, dtype=torch.uint8, device="cuda"),
+                  sums=torch.empty(nb, dtype=torch.float64, device="cuda"))
+        wsb = int(sb.lib.sbsa_select_workspace_bytes(ctypes.byref(ps)))
+        st["ws"], st["wsb"] = torch.empty(wsb, dtype=torch.uint8, device="cuda"), wsb
+        st["args"] = (ctypes.byref(ps), sb._ptr(st["qc"]), sb._ptr(st["kc"]), None,
+                      sb._ptr(st["idx"]), sb._ptr(st["cnt"]), sb._ptr(st["flags"]),
+                      sb._ptr(st["ws"]), wsb)
+        assert sb.lib.sbsa_select_gate_partial(*st["args"], sb._ptr(st["sums"]), None) == sb.OK
+        shards.append(st)
+    for st in shards:
+        sums += st["sums"]
+    for st in shards:
+        assert sb.lib.sbsa_select_gate_finish(*st["args"], sb._ptr(sums), w.n_sel_heads,
+                                              None) == sb.OK
+    torch.cuda.synchronize()
+    assert sb.get_status() == sb.OK
+    idx = torch.cat([st["idx"] for st in shards]).cpu().numpy()
+    cnt = torch.cat([st["cnt"] for st in shards]).cpu().numpy()
+    budgets = _budgets(w, ref)
+    exact, tie = PT.compare_lists(idx, cnt, ref["idx"], ref["cnt"], _all_rows(w), ref["qbar"],
+                                  ref["c"], ref["r"], w, _kv_of_sel(w), minmax=ref["minmax"],
+                                  budgets=budgets)
+    PT.record("gate_two_shards", name, rows=exact + tie, exact=exact, tie=tie,
+              sigma_band_tiles=PT.sigma_band_tiles(budgets))
+    assert tie <= max(2, 0.01 * (exact + tie)), (exact, tie)
+    # tiles with at most k candidates carry no margin
+    assert int(torch.isnan(sums).sum()) == w.top_k + 1
+
+
 def test_gate_fires_on_the_planted_rows(sb):
     w, data, ref = small_case("gate_small")
     p = sb.params_for(w)

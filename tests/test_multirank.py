@@ -148,3 +148,93 @@ def test_gpus_beyond_the_visible_devices_fails_loudly():
     rc, line, err = _bench("--gpus", "4096", "--launch-check")
     assert rc != 0 and line is None
     assert "visible" in err
+
+
+# ------------------------------------- percentile gate across head shards
+
+def _gate_shard_worker(rank, world, port, name, out):
+    """One rank of a sequence sharded by kv head under the percentile gate:
+    the oracle's cut margins of this rank's selection heads, summed per tile,
+    all-reduced over the ranks, then the tile decisions and this rank's lists."""
+    import math
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    import oracle as O
+    from block_sparse_attention_sbsa_b200 import workloads as W
+    w = W.SMALL[name]
+    data = W.generate(w, "cpu")
+    ws, (g0, g1) = bench.shard_workload(w, rank, world)
+    d = bench.shard_tensors(data, w, g0, g1)
+    ks = d["k_idx"] if ws.index_dim else d["k"]
+    qs = d["q_idx"] if ws.index_dim else d["q"]
+    c, r = O.pool_keys(ks, ws.block_size, with_radius=False)
+    r = np.zeros(c.shape[:2])
+    mm = O.pool_keys_minmax(ks, ws.block_size) if ws.backbone == "minmax" else None
+    qbar = O.pool_queries(qs, ws.block_size, group=1)
+    scale = 1.0 / math.sqrt(ws.score_dim)
+    kv = lambda hs: hs // ws.group
+    nb, k = ws.n_blocks, ws.top_k
+
+    def scores(h, i):
+        if mm is None:
+            return O.block_scores(qbar[h, i], c[kv(h)], i, scale)
+        return O.block_bounds_minmax(qbar[h, i], mm[0][kv(h)], mm[1][kv(h)], i, scale)
+    sums = torch.zeros(nb, dtype=torch.float64)
+    for i in range(k + 1, nb):
+        tot = 0.0
+        for h in range(ws.n_sel_heads):            # this rank's heads, head order
+            tot += O.cut_margin(scores(h, i), k)
+        sums[i] = tot
+    dist.all_reduce(sums)                          # the one exchange of the path
+    total = w.n_sel_heads
+    sbar = {i: float(sums[i]) / total for i in range(k + 1, nb)}
+    q = float(np.float32(w.gate_quantile))
+    fired = O.percentile_fire(sbar, q)
+    idx, cnt, _ = O.select(qbar, c, r, block_count=nb, mode=ws.select_mode, top_k_=k,
+                           scale=scale, kv_of_sel=kv, max_blocks=ws.max_blocks, minmax=mm,
+                           sigma_gate=(q, w.gate_rho), fired=fired)
+    out[rank] = (g0, g1, sorted(fired), sbar, idx, cnt)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name", ["sigma_small", "sigma_quest_small"])
+def test_percentile_gate_decomposes_over_head_shards_with_one_all_reduce(name):
+    """The percentile gate couples heads (a tile's mean margin over all
+    selection heads).  Two ranks, each holding half the kv heads, reproduce the
+    unsharded oracle's fired tiles and lists after one all-reduce of their
+    per-tile margin sums."""
+    import numpy as np
+    import oracle as O
+    import parity as PT
+    from block_sparse_attention_sbsa_b200 import workloads as W
+    world, port = 2, _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_gate_shard_worker, args=(world, port, name, out), nprocs=world, join=True)
+    w = W.SMALL[name]
+    data = W.generate(w, "cpu")
+    q = float(np.float32(w.gate_quantile))
+    full = O.prefill(data["q"], data["k"], data["v"], block=w.block_size, mode=w.select_mode,
+                     top_k_=w.top_k, max_blocks=w.max_blocks, backbone=w.backbone,
+                     sigma_gate=(q, w.gate_rho))
+    fired0, fired1 = out[0][2], out[1][2]
+    assert fired0 == fired1                          # both ranks decided alike
+    # the ranks' sums add in another order than one head-order sum: every
+    # tile's decision agrees with the unsharded one outside SIGMA_BAND
+    budgets = PT.percentile_budgets(full["sbar"], full["fired"], w.top_k, w.gate_rho)
+    for i, b in budgets.items():
+        took = w.gate_rho * w.top_k if i in fired0 else w.top_k
+        assert took in b, i
+        assert abs(out[0][3][i] - full["sbar"][i]) < 1e-12
+    for rank in range(world):
+        g0, g1 = out[rank][0], out[rank][1]
+        hs0, hs1 = g0 * w.group, g1 * w.group
+        if set(fired0) == set(full["fired"]):
+            assert np.array_equal(out[rank][4], full["idx"][hs0:hs1])
+            assert np.array_equal(out[rank][5], full["cnt"][hs0:hs1])
