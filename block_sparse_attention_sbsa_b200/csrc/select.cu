@@ -41,6 +41,7 @@ namespace {
 constexpr int kSelThreads = 256;
 constexpr int kWarps = kSelThreads / 32;
 constexpr int kMaxWalk = 24;  // ranked-walk steps before the radix fallback
+constexpr int kShortWalk = 4;  // rank keys per lane kept for the walk
 constexpr int kHistBytes = kWarps * 256 * 8;  // one 256-bin 64-bit histogram per warp
 constexpr int kShortCap = 256;                // short-list keys (second half of a warp's area)
 
@@ -511,14 +512,41 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
       if (n == 0) {
         select_all = true;
       } else {
-        // four independent partials per lane keep four loads in flight
+        // four independent partials per lane keep four loads in flight; the
+        // same pass keeps each lane's kShortWalk largest rank keys (descending)
+        // for the walk below, inserting only candidates that reach the
+        // lane's current smallest kept score
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        uint64_t top[kShortWalk];
+#pragma unroll
+        for (int q = 0; q < kShortWalk; ++q) top[q] = 0ull;
+        float floor_s = -INFINITY;
+        auto keep = [&](float sv, int jx) {
+          if (sv >= floor_s) {
+            uint64_t c = rank_key(sv, jx);
+#pragma unroll
+            for (int q = 0; q < kShortWalk; ++q) {
+              const uint64_t hi = c > top[q] ? c : top[q];
+              c = c > top[q] ? top[q] : c;
+              top[q] = hi;
+            }
+            if (top[kShortWalk - 1]) floor_s = key_float((uint32_t)(top[kShortWalk - 1] >> 32));
+          }
+        };
         int j = lane;
         for (; j + 96 < n; j += 128) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) m4[u] = fmaxf(m4[u], s[j + 32 * u]);
+          for (int u = 0; u < 4; ++u) {
+            const float sv = s[j + 32 * u];
+            m4[u] = fmaxf(m4[u], sv);
+            keep(sv, j + 32 * u);
+          }
         }
-        for (; j < n; j += 32) m4[0] = fmaxf(m4[0], s[j]);
+        for (; j < n; j += 32) {
+          const float sv = s[j];
+          m4[0] = fmaxf(m4[0], sv);
+          keep(sv, j);
+        }
         const float m = warp_max_f(fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
         double z4[4] = {0.0, 0.0, 0.0, 0.0};
         j = lane;
@@ -535,7 +563,33 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
         // same order as the definition (descending score, lower id first).
         uint64_t prev = ~0ull, cum = 0;
         int taken = 0;
-        for (; taken < kMaxWalk && taken < n; ++taken) {
+        // First on the lanes' short lists: the next key of the ranked order is
+        // the largest lane head, as long as no lane has used up its short list
+        // while holding further candidates (whose keys it did not keep).
+        {
+          const int mine = lane < n ? (n - 1 - lane) / 32 + 1 : 0;  // this lane's candidates
+          int used = 0;
+          for (; taken < kMaxWalk && taken < n; ++taken) {
+            const bool blind = used == kShortWalk && mine > kShortWalk;
+            if (__any_sync(0xFFFFFFFFu, blind)) break;
+            const uint64_t head = top[0];
+            const uint64_t best = warp_max_u64(head);
+            if (head == best) {  // keys are unique: one lane moves on
+#pragma unroll
+              for (int q = 0; q + 1 < kShortWalk; ++q) top[q] = top[q + 1];
+              top[kShortWalk - 1] = 0ull;
+              ++used;
+            }
+            prev = best;
+            cum += mass_weight(key_float((uint32_t)(best >> 32)), m, wscale);
+            if (cum >= want) {
+              walked = true;
+              break;
+            }
+          }
+        }
+        // then, if needed, one maximum at a time over the whole row
+        for (; !walked && taken < kMaxWalk && taken < n; ++taken) {
           uint64_t b4[4] = {0, 0, 0, 0};
           int jj = lane;
           for (; jj + 96 < n; jj += 128) {
@@ -602,6 +656,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
     // loads), then the chunks are emitted in order.
     int written = 0, tie_seen = 0;
     bool rescued_extra = false;
+    // The cut as a float: for non-NaN scores, fkey(x) > fkey(c) exactly when
+    // x > c and fkey(x) == fkey(c) when x == c (-0 and +0 alike), so the
+    // per-candidate tests need no keys.  A walked cut also carries its block
+    // id: rank_key(x, j) >= wkey is x > c, or x == c with j <= the cut's id.
+    const float cut = walked ? key_float((uint32_t)(wkey >> 32)) : key_float(vkey);
+    const int cut_id = walked ? (int)(0xFFFFFFFFu - (uint32_t)wkey) : 0;
     for (int base = 0; base < n; base += 128) {
       bool bsel[4], eqk[4], resc[4];
 #pragma unroll
@@ -615,11 +675,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
           if (select_all) {
             bsel[u] = true;
           } else if (walked) {
-            bsel[u] = rank_key(sj, j) >= wkey;
+            bsel[u] = sj > cut || (sj == cut && j <= cut_id);
           } else {
-            const uint32_t k = fkey(sj);
-            bsel[u] = k > vkey;
-            eqk[u] = k == vkey;
+            bsel[u] = sj > cut;
+            eqk[u] = sj == cut;
           }
           if (a.rescue) resc[u] = fmaf(qn_s, krs[j], sj) > a.tau;
         }
