@@ -23,6 +23,7 @@ SOURCES = ["pool.cu", "select.cu", "score_rowmax.cu", "score_centroid.cu", "atte
            "attend_ps64.cu",
            "attend_pair.cu",
            "sbsa_api.cu",
+           "sbsa_host.cu",
            "sbsa_noalloc.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "tma_map.h"]
 

@@ -151,4 +151,7 @@ cudaError_t launch_wait_probe(uint64_t timeout_ns, int* status, cudaStream_t str
 // Device status word of the current device (recorded by kernels).
 int* device_status_ptr();
 
+// The argument checks every entry point makes (SBSA_OK or an error code).
+int validate_params(const sbsa_params* p);
+
 }  // namespace sbsa

@@ -106,6 +106,12 @@ int validate(const sbsa_params* p, Derived* d) {
   return SBSA_OK;
 }
 
+}  // namespace
+
+int validate_params(const sbsa_params* p) { return validate(p, nullptr); }
+
+namespace {
+
 int attend_supported(const sbsa_params* p) {
   if (p->dtype == SBSA_FP32 && !(p->head_dim == 64 && p->block_size == 64))
     return SBSA_ERR_UNSUPPORTED;

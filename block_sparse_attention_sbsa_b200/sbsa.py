@@ -31,7 +31,7 @@ SYMBOLS = ["sbsa_pool_blocks", "sbsa_pool_minmax", "sbsa_select", "sbsa_select_w
            "sbsa_score_centroids_workspace_bytes", "sbsa_score_rowmax",
            "sbsa_score_rowmax_workspace_bytes",
            "sbsa_select_scores", "sbsa_select_gate_partial", "sbsa_select_gate_finish",
-           "sbsa_attend", "sbsa_prefill",
+           "sbsa_attend", "sbsa_prefill", "sbsa_prefill_host", "sbsa_prefill_host_workspace_bytes",
            "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string",
            "sbsa_version", "sbsa_debug_wait_timeout"]
 
@@ -111,6 +111,9 @@ def _load() -> ctypes.CDLL:
     lib.sbsa_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i32p, i32p, u8p, vp]
     lib.sbsa_prefill_workspace_bytes.argtypes = [P]
     lib.sbsa_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.sbsa_prefill_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.sbsa_prefill_host_workspace_bytes.argtypes = [P]
+    lib.sbsa_prefill_host_workspace_bytes.restype = ctypes.c_size_t
     lib.sbsa_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.sbsa_status_string.argtypes = [ci]
     lib.sbsa_status_string.restype = ctypes.c_char_p
@@ -371,6 +374,38 @@ class Prefill:
                                 _ptr(k_idx) if p.index_dim else None, _ptr(out), _ptr(self.ws),
                                 self.ws.numel(), _ptr(self.idx), _ptr(self.cnt), _ptr(self.flags),
                                 _stream(stream)), "sbsa_prefill")
+        return out
+
+
+class PrefillHost:
+    """Reusable prefill from host tensors to a host output through
+    sbsa_prefill_host (one C call per request; the library pipelines the
+    copies and the computation over chunks of kv heads).  Host tensors
+    should be pinned; they must stay untouched until the stream has
+    completed the request."""
+
+    def __init__(self, p: Params, device="cuda"):
+        self.p = p
+        n = int(lib.sbsa_prefill_host_workspace_bytes(ctypes.byref(p)))
+        if n == 0:
+            raise SbsaError(ERR_INVALID_ARG, "sbsa_prefill_host_workspace_bytes")
+        self.ws = torch.empty(n, device=device, dtype=torch.uint8)
+
+    def __call__(self, q, k, v, out, q_idx=None, k_idx=None, stream=None):
+        p = self.p
+        dt = _TORCH_DT[p.dtype]
+        for t, name, shape in ((q, "q", (p.n_q_heads, p.seq_len, p.head_dim)),
+                               (k, "k", (p.n_kv_heads, p.seq_len, p.head_dim)),
+                               (v, "v", (p.n_kv_heads, p.seq_len, p.head_dim)),
+                               (out, "out", (p.n_q_heads, p.seq_len, p.head_dim))):
+            if t.device.type != "cpu" or t.dtype != dt or tuple(t.shape) != shape \
+                    or not t.is_contiguous():
+                raise ValueError(f"{name}: expected a contiguous host {dt} tensor of {shape}")
+        _check(lib.sbsa_prefill_host(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(q_idx) if p.index_dim else None,
+                                     _ptr(k_idx) if p.index_dim else None, _ptr(out),
+                                     _ptr(self.ws), self.ws.numel(), _stream(stream)),
+               "sbsa_prefill_host")
         return out
 
 

@@ -313,6 +313,34 @@ int sbsa_prefill(const sbsa_params* p, const void* q, const void* k, const void*
                  size_t ws_bytes, int32_t* idx_out, int32_t* cnt_out, uint8_t* flags_out,
                  void* stream);
 
+/*
+ * sbsa_prefill_host -- sbsa_prefill from and to HOST memory.  The pages have
+ * no such call; it is the end-to-end form of the prefill for a caller whose
+ * tensors live on the host.
+ *   q, k, v, q_idx, k_idx: host, layouts as in sbsa_prefill (page-locked
+ *                memory lets the copies overlap the computation; pageable
+ *                memory is correct but the copies then wait for the host).
+ *   o:           host [Hq, N, d] out, written when the call's work on
+ *                `stream` completes.
+ *   workspace:   device, 256-byte aligned, ws_bytes >=
+ *                sbsa_prefill_host_workspace_bytes(p): two staging sets of one
+ *                chunk's inputs and output, and the chunk prefill's workspace.
+ * The request is cut into chunks of kv heads (each kv head with the query
+ * heads that read it; one chunk under the percentile gate, which averages
+ * over every head): chunk c + 1 is copied in while chunk c is prefilled on
+ * `stream` and chunk c - 1 is copied out.  The copies run on two streams of
+ * the library's own per device, created on the first call (make that call
+ * before any stream capture), ordered after the work already on `stream`;
+ * everything the call enqueues is complete once `stream` reaches its end.
+ * Calls that overlap on one device share those copy streams and run in turn.
+ * Lists are not returned (they stay in the workspace).  Errors as
+ * sbsa_prefill.
+ */
+size_t sbsa_prefill_host_workspace_bytes(const sbsa_params* p);
+int sbsa_prefill_host(const sbsa_params* p, const void* q, const void* k, const void* v,
+                      const void* q_idx, const void* k_idx, void* o, void* workspace,
+                      size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the current device's status
  * word into *device_status (SBSA_OK when no kernel reported an error).
  * Returns SBSA_ERR_CUDA when the synchronisation itself failed. */

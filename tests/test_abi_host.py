@@ -283,6 +283,29 @@ def test_shared_memory_limits_are_rejected_before_launch(sb, kw, ok_len, bad_len
                                1 << 40, None, None, None, None) == 2
 
 
+def test_prefill_host_workspace_and_checks(sb):
+    p = _valid(sb, seq_len=4096)                    # 4 query / 2 kv heads: two chunks
+    need = sb.lib.sbsa_prefill_host_workspace_bytes(ctypes.byref(p))
+    sub = _valid(sb, seq_len=4096, n_q_heads=2, n_kv_heads=1)
+    n, d = 4096, 128
+    q_chunk, kv_chunk = r256(2 * n * d * 2), r256(n * d * 2)
+    staging = q_chunk + 2 * kv_chunk + q_chunk        # Q, K, V and O of one chunk
+    assert need == 2 * staging + r256(sb.workspace_bytes(sub))
+    f = sb.lib.sbsa_prefill_host
+    assert f(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, FAKE, FAKE, need - 1, None) == 3
+    assert f(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, FAKE,
+             ctypes.c_void_p((1 << 20) + 128), need, None) == 3
+    assert f(ctypes.byref(p), FAKE, None, FAKE, None, None, FAKE, FAKE, need, None) == 1
+    bad = _valid(sb, head_dim=96)
+    assert f(ctypes.byref(bad), FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 40, None) == 2
+    assert sb.lib.sbsa_prefill_host_workspace_bytes(ctypes.byref(bad)) == 0
+    # the percentile gate couples heads: one chunk holding every head
+    g = _valid(sb, seq_len=4096, gate_quantile=0.3, gate_rho=2)
+    one = r256(4 * n * d * 2) * 2 + r256(2 * n * d * 2) * 2
+    assert sb.lib.sbsa_prefill_host_workspace_bytes(ctypes.byref(g)) == \
+        2 * one + r256(sb.workspace_bytes(g))
+
+
 def test_fp32_attention_is_limited_to_d64_b64(sb):
     p = _valid(sb, dtype="fp32")
     assert _attend(sb, p) == 2

@@ -565,6 +565,28 @@ def test_degenerate_selection_parameters(sb, case):
     assert mx <= PT.MAX_ABS and mean <= PT.MEAN_ABS, (mx, mean)
 
 
+@pytest.mark.parametrize("name", ["gqa_small", "msa_small", "sigma_small", "tiny"])
+def test_prefill_host_equals_the_device_prefill(sb, name):
+    """sbsa_prefill_host (host tensors in and out, pipelined over chunks of kv
+    heads; index tensors for the group-shared workload; one chunk under the
+    percentile gate; fp32) gives the device prefill's output exactly, on two
+    requests in a row."""
+    w, data, ref = small_case(name)
+    p = sb.params_for(w)
+    d = _dev(data)
+    o_dev, _, _, _ = sb.prefill(p, d["q"], d["k"], d["v"], d["q_idx"], d["k_idx"])
+    torch.cuda.synchronize()
+    host = {k: data[k].contiguous().pin_memory() for k in ("q", "k", "v", "q_idx", "k_idx")
+            if data[k] is not None}
+    call = sb.PrefillHost(p)
+    for _ in range(2):
+        out = torch.zeros(data["q"].shape, dtype=data["q"].dtype).pin_memory()
+        call(host["q"], host["k"], host["v"], out, host.get("q_idx"), host.get("k_idx"))
+        torch.cuda.synchronize()
+        assert sb.get_status() == sb.OK
+        assert torch.equal(out, o_dev.cpu())
+
+
 def test_prefill_pipeline_from_host_buffers(sb):
     """PrefillPipeline: pinned host inputs -> device -> prefill -> pinned host
     output, three requests in flight order, each equal to a plain prefill."""
