@@ -436,17 +436,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
         tmem_ld32(s_col + hf * 64 + 32, bb);
         tmem_wait_ld();
         const int c0 = hf * 64;  // key index of a[0] within the block
-        float mx = -INFINITY;
         if (diag) {
+          // causal mask of the diagonal block: keys past the row's own token
+          // score -inf, so the maximum and the exponentials below need no
+          // test of their own (exp2(-inf) = +0)
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            if (c0 + c <= row) mx = fmaxf(mx, a[c]);
-            if (c0 + 32 + c <= row) mx = fmaxf(mx, bb[c]);
+            if (c0 + c > row) a[c] = -INFINITY;
+            if (c0 + 32 + c > row) bb[c] = -INFINITY;
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(a[c], bb[c]));
         }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(a[c], bb[c]));
         // exchange the half-row maxima with the partner warp; both warps have
         // finished reading S, so P may then overwrite the first S columns
         float* mxb = mx_buf + (g & 1) * 2 * BM;
@@ -491,12 +493,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
           float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
           float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
           float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
-          if (diag) {
-            if (c0 + c > row) p0 = 0.f;
-            if (c0 + c + 1 > row) p1 = 0.f;
-            if (c0 + 32 + c > row) p2 = 0.f;
-            if (c0 + 32 + c + 1 > row) p3 = 0.f;
-          }
           lsum += (p0 + p1) + (p2 + p3);
           pk[c >> 1] = pack_bf16x2(p0, p1);
           pk[16 + (c >> 1)] = pack_bf16x2(p2, p3);

@@ -468,9 +468,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
         float a[32];
         tmem_ld32(s_col + c0, a);
         tmem_wait_ld();
+        const bool active = jh >= 0;  // uniform across the warp (one half)
+        if (active && lim < 31) {
+          // the diagonal block: keys past lim score -inf, so neither the
+          // maximum nor the exponentials need a test (exp2(-inf) = +0)
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c > lim) a[c] = -INFINITY;
+        }
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, c <= lim ? a[c] : -INFINITY);
+        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, a[c]);
         // exchange the half-row maxima with the partner warp; both warps have
         // finished reading S, so P may then overwrite the first S columns
         float* mxb = mx_buf + (g & 1) * 2 * BM;
@@ -481,7 +489,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
           ok = false;
           break;
         }
-        const bool active = jh >= 0;  // uniform across the warp (one half)
         if (active) {
           mx = fmaxf(mx, mxb[(hf ^ 1) * BM + row]);
           const float m_new = fmaxf(m_run, mx * p.scale_log2);
@@ -510,18 +517,23 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
           }
         }
         // P = exp2(S * scale - m) as bf16 over this warp's 32 keys -> columns
-        // [c0/2, c0/2 + 16); zeros over 16 columns of the other half's keys
+        // [c0/2, c0/2 + 16), zeros when the half is idle (its running maximum
+        // may still be -inf); zeros over 16 columns of the other half's keys
         float lsum = 0.f;
         uint32_t pk[16], zero[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
-          float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
-          p0 = c <= lim ? p0 : 0.f;
-          p1 = c + 1 <= lim ? p1 : 0.f;
-          lsum += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-          zero[c >> 1] = 0u;
+        for (int c = 0; c < 16; ++c) zero[c] = 0u;
+        if (active) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
+            const float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
+            lsum += p0 + p1;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pk[c] = 0u;
         }
         tmem_st16u(s_col + (c0 >> 1), pk);
         tmem_st16u(s_col + (1 - half) * 32 + hf * 16, zero);
