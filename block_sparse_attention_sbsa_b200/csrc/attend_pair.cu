@@ -519,27 +519,32 @@ __global__ void __launch_bounds__(kThreads, 1) attend_pair_kernel(const __grid_c
           }
         }
         // pass 2: P = exp2(S * scale - m) as bf16 over the first half of the
-        // S columns (step c0 reads S[c0, c0+64), writes P to [c0/2, c0/2+32))
+        // S columns (step c0 reads S[c0, c0+64), writes P to [c0/2, c0/2+32));
+        // the two steps stay a loop: unrolled, the kernel spills
         float lsum = 0.f;
-#pragma unroll
+#pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 64) {
           float a[32], bb[32];
           tmem_ld32(s_col + c0, a);
           tmem_ld32(s_col + c0 + 32, bb);
           tmem_wait_ld();
+          if (diag) {
+            // causal mask of the diagonal block: keys past the row's own
+            // token score -inf, so the exponentials need no test of their
+            // own (exp2(-inf) = +0)
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (c0 + c > row) a[c] = -INFINITY;
+              if (c0 + 32 + c > row) bb[c] = -INFINITY;
+            }
+          }
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
-            float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
-            float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
-            float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
-            if (diag) {
-              if (c0 + c > row) p0 = 0.f;
-              if (c0 + c + 1 > row) p1 = 0.f;
-              if (c0 + 32 + c > row) p2 = 0.f;
-              if (c0 + 32 + c + 1 > row) p3 = 0.f;
-            }
+            const float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
+            const float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
+            const float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
+            const float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
             lsum += (p0 + p1) + (p2 + p3);
             pk[c >> 1] = pack_bf16x2(p0, p1);
             pk[16 + (c >> 1)] = pack_bf16x2(p2, p3);
