@@ -34,6 +34,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace sbsa {
 namespace {
@@ -44,6 +45,7 @@ constexpr int kMaxWalk = 24;  // ranked-walk steps before the radix fallback
 constexpr int kShortWalk = 4;  // rank keys per lane kept for the walk
 constexpr int kHistBytes = kWarps * 256 * 8;  // one 256-bin 64-bit histogram per warp
 constexpr int kShortCap = 256;                // short-list keys (second half of a warp's area)
+constexpr uint64_t kStageTimeoutNs = 2000000000ull;  // bound on the staging copies' wait
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
@@ -318,14 +320,60 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
     if (!__syncthreads_or(any)) return;
   }
 
-  for (int e = tid; e < R * DS; e += kSelThreads) {
-    const int r = e / DS;
-    qs[e] = (r < rows && a.qc) ? a.qc[((size_t)hs * a.nb + i0 + r) * DS + (e % DS)] : 0.f;
-  }
-  if (a.rescue) {
-    // the kv head's radii of every candidate, read once per CTA
-    const float* kr = a.kr + (size_t)g * a.nb;
-    for (int j = tid; j < jend; j += kSelThreads) krs[j] = kr[j];
+  // ---- staging: the rows' pooled queries, the kv head's radii of every
+  // candidate (rescue) and, from a precomputed table, the rows' scores.  When
+  // every source is 16-byte aligned, thread 0 issues them as bulk copies on
+  // one barrier (one memory round trip for the whole CTA); otherwise the
+  // threads copy them.
+  __shared__ __align__(8) uint64_t stage_bar;
+  const float* const score_base = a.scores ? a.scores + ((size_t)hs * a.nb + i0) * a.nb : nullptr;
+  const bool bulk = a.qc && (reinterpret_cast<uintptr_t>(a.qc) & 15) == 0 && (a.nb & 3) == 0 &&
+                    (!a.rescue || (reinterpret_cast<uintptr_t>(a.kr) & 15) == 0) &&
+                    (!a.scores || (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0);
+  if (bulk) {
+    if (tid == 0) {
+      mbar_init(&stage_bar, 1);
+      fence_barrier_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+      // candidates rounded up to whole 16-byte pieces; nb is a multiple of 4,
+      // so no row is read past its end
+      const uint32_t q_bytes = (uint32_t)(rows * DS * 4);
+      const uint32_t r_bytes = a.rescue ? (uint32_t)(((jend + 3) & ~3) * 4) : 0u;
+      uint32_t total = q_bytes + r_bytes;
+      if (score_base)
+        for (int r = 0; r < rows; ++r) total += (uint32_t)(((i0 + r + 3) & ~3) * 4);
+      mbar_arrive_expect_tx(&stage_bar, total);
+      bulk_load(qs, a.qc + ((size_t)hs * a.nb + i0) * DS, q_bytes, &stage_bar);
+      if (r_bytes) bulk_load(krs, a.kr + (size_t)g * a.nb, r_bytes, &stage_bar);
+      if (score_base) {
+        for (int r = 0; r < rows; ++r) {
+          const uint32_t b = (uint32_t)(((i0 + r + 3) & ~3) * 4);
+          if (b) bulk_load(sc + (size_t)r * score_stride, score_base + (size_t)r * a.nb, b, &stage_bar);
+        }
+      }
+    }
+    for (int e = rows * DS + tid; e < R * DS; e += kSelThreads) qs[e] = 0.f;
+    volatile int never = 0;
+    const bool landed = mbar_wait_bounded(&stage_bar, 0, &never, kStageTimeoutNs);
+    if (__syncthreads_or(!landed)) {
+      // the copies did not land in time: report it, let them finish (with a
+      // bound) before the CTA's shared memory is released, and skip the rows
+      if (tid == 0) record_status(a.status, SBSA_ERR_TIMEOUT);
+      mbar_wait_bounded(&stage_bar, 0, &never, kStageTimeoutNs);
+      return;
+    }
+  } else {
+    for (int e = tid; e < R * DS; e += kSelThreads) {
+      const int r = e / DS;
+      qs[e] = (r < rows && a.qc) ? a.qc[((size_t)hs * a.nb + i0 + r) * DS + (e % DS)] : 0.f;
+    }
+    if (a.rescue) {
+      // the kv head's radii of every candidate, read once per CTA
+      const float* kr = a.kr + (size_t)g * a.nb;
+      for (int j = tid; j < jend; j += kSelThreads) krs[j] = kr[j];
+    }
   }
   __syncthreads();
 
@@ -333,10 +381,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
   // and streams their centroid rows (fp32) from L2 in 16-byte pieces, dotting
   // each piece with the R pooled queries read from shared memory (every lane
   // reads the same address: one broadcast per row).
-  if (a.scores) {
+  if (a.scores && !bulk) {
     // precomputed scores (centroid or row-max): copy the rows' candidates,
     // four rows' loads in flight per thread
-    const float* base = a.scores + ((size_t)hs * a.nb + i0) * a.nb;
+    const float* base = score_base;
     if ((a.nb & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0) {
       for (int r0 = 0; r0 < rows; r0 += 4) {
         for (int j4 = tid; 4 * j4 < i0 + r0 + 3; j4 += kSelThreads) {
@@ -362,7 +410,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
         for (int j = tid; j < i0 + r; j += kSelThreads) sc[r * score_stride + j] = src[j];
       }
     }
-  } else if (a.minmax) {
+  } else if (!a.scores && a.minmax) {
     // Upper-bound backbone: s_j = sum_d max(q_d min_jd, q_d max_jd), the two
     // table rows of block j streamed like a centroid row.
     const float* km = a.kc + (size_t)g * a.nb * 2 * DS;
@@ -788,8 +836,12 @@ size_t select_smem(int rows, int nb, int ds, int rescue) {
 
 template <int DS>
 cudaError_t launch_ds(const SelectArgs& a, cudaStream_t stream) {
-  // rows per CTA: as many (up to 16) as the score rows allow in shared memory;
-  // more rows per CTA means fewer reads of each centroid row from L2
+  // rows per CTA.  Scores read from a precomputed table: 8, so that three
+  // CTAs (24 warps) fit an SM and hide the per-row latency.  Scores computed
+  // here: as many (up to 16) as the score rows allow in shared memory, since
+  // more rows per CTA means fewer reads of each centroid row from L2.
+  if (a.scores && select_smem(8, a.nb, DS, a.rescue) <= kSelectBudget)
+    return launch_rows<DS, 8>(a, stream);
   if (select_smem(16, a.nb, DS, a.rescue) <= kSelectBudget) return launch_rows<DS, 16>(a, stream);
   if (select_smem(8, a.nb, DS, a.rescue) <= kSelectBudget) return launch_rows<DS, 8>(a, stream);
   if (select_smem(4, a.nb, DS, a.rescue) <= kSelectBudget) return launch_rows<DS, 4>(a, stream);
