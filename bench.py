@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 NCU_ATTEND_TRAFFIC = {
     # profiles/attend_ps_kernel_dram_rbs.md: 2.36 GB read + 1.05 GB written
     "rbs128k": {"bytes": 3.41e9, "source": "block_sparse_attention_sbsa_b200/csrc/attend_persist.cu",
-                "sha": "f341cf8598eab1c7"},
+                "sha": "6bb6ffa558abafcc"},
 }
 
 

@@ -23,8 +23,10 @@
 //                        first half of S[g % 2], where the softmax wrote it.
 //   warps 2-9  softmax: two warps per TMEM lane quadrant, each owning 64 of
 //              the 128 key columns of its 32 query rows; the row maximum is
-//              exchanged through shared memory (a 64-arrival mbarrier per
-//              quadrant, bounded wait), the running maximum is moved (and O rescaled in
+//              exchanged through shared memory at a named barrier of the two
+//              warps (which also tells both whether either has failed a
+//              bounded wait, so they leave together), the running maximum is
+//              moved (and O rescaled in
 //              TMEM, each warp its half of the columns) only when it grows
 //              by more than 2^8; P is written back as bf16; the two partial
 //              row sums are handed to the epilogue per item.
@@ -62,8 +64,8 @@ struct PS {
   static constexpr int OFF_MX = OFF_L + 4 * BM * 4;          // row max [block%2][half][BM]
   static constexpr int OFF_BAR = OFF_MX + 4 * BM * 4;
   // q_full[2] q_free[2] kv_full[S] s_full[2] p_full[2] pv_done[2]
-  // o_full[2] o_free[2] l_full[2] mx_ready[2][4] drain
-  static constexpr int NBARS = 2 + 2 + kStages + 2 + 2 + 2 + 2 + 2 + 2 + 8 + 1;
+  // o_full[2] o_free[2] l_full[2] drain
+  static constexpr int NBARS = 2 + 2 + kStages + 2 + 2 + 2 + 2 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S = 0;       // S[0], S[1]: 2 x BN columns
@@ -167,8 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
   uint64_t* o_full = pv_done + 2;
   uint64_t* o_free = o_full + 2;
   uint64_t* l_full = o_free + 2;
-  uint64_t* mx_ready = l_full + 2;  // [block % 2][quadrant]
-  uint64_t* drain = mx_ready + 8;
+  uint64_t* drain = l_full + 2;
   float* l_buf = reinterpret_cast<float*>(smem + C::OFF_L);
   float* mx_buf = reinterpret_cast<float*>(smem + C::OFF_MX);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -189,7 +190,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
       mbar_init(&o_full[b], 1);
       mbar_init(&o_free[b], 128);
       mbar_init(&l_full[b], 256);
-      for (int q = 0; q < 4; ++q) mbar_init(&mx_ready[b * 4 + q], 64);
     }
     for (int s = 0; s < kStages; ++s) mbar_init(&kv_full[s], 1);
     mbar_init(drain, 1);
@@ -343,6 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
     for (; ok && load_item(p, t, it, lane); ++t) {
       const int qb = t & 1;
       bool good = true;
+      // The warp reads the item's list together (load_item); lane 0 alone
+      // waits and issues for the item's blocks (one per valid entry, in list
+      // order, as the producer loads them), and the outcome reaches the warp
+      // once per item.
       if (lane == 0) {
         good = wait(&q_full[qb], (t >> 1) & 1);
         if (good) {
@@ -353,18 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
             umma_commit(&o_full[qb]);
           }
         }
-      }
-      if (!warp_ok(good)) {
-        ok = false;
-        break;
-      }
-      if (it.valid == 0) continue;
-      int b = 0;
-      for (int r = 0; r < it.count; ++r) {
-        const int j = item_entry(it, r, lane);
-        if (!valid_entry(it, j)) continue;
-        const bool last = (b == it.valid - 1);
-        if (lane == 0) {
+        for (int b = 0; good && b < it.valid; ++b) {
+          const bool last = (b == it.valid - 1);
           const int kpos = 2 * g;
           const int st = kpos % kStages;
           good = wait(&kv_full[st], (kpos / kStages) & 1);
@@ -386,15 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
             if (last) umma_commit(&q_free[qb]);
             if (have_prev) good = issue_pv(prev);
           }
+          prev = Pending{g, t, b, last ? 1 : 0};
+          have_prev = true;
+          ++g;
         }
-        if (!warp_ok(good)) {
-          ok = false;
-          break;
-        }
-        prev = Pending{g, t, b, last ? 1 : 0};
-        have_prev = true;
-        ++g;
-        ++b;
+      }
+      if (!warp_ok(good)) {
+        ok = false;
+        break;
       }
     }
     if (lane == 0) {
@@ -424,11 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
         if (!valid_entry(it, j)) continue;
         const bool diag = (j == it.i);
         const uint32_t s_col = tmem + lane_base + C::TM_S + (g & 1) * BN;
-        if (!wait(&s_full[g & 1], (g >> 1) & 1)) ok = false;
-        if (!__all_sync(0xFFFFFFFFu, ok)) {
-          ok = false;
-          break;
-        }
+        const bool s_ok = __all_sync(0xFFFFFFFFu, wait(&s_full[g & 1], (g >> 1) & 1));
         tc_fence_after();
         // this warp's 64 S columns, kept in registers
         float a[32], bb[32];
@@ -453,9 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
         // finished reading S, so P may then overwrite the first S columns
         float* mxb = mx_buf + (g & 1) * 2 * BM;
         mxb[hf * BM + row] = mx;
-        mbar_arrive(&mx_ready[(g & 1) * 4 + qd]);
-        if (!wait(&mx_ready[(g & 1) * 4 + qd], (g >> 1) & 1)) ok = false;
-        if (!__all_sync(0xFFFFFFFFu, ok)) {
+        // the two warps of the quadrant meet once per block; the barrier also
+        // tells both whether either missed its S, so they leave together
+        if (bar_red_or(1 + qd, 64, !s_ok)) {
           ok = false;
           break;
         }
@@ -464,9 +453,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
         if (b == 0) {
           m_run = m_new;
         } else if (__any_sync(0xFFFFFFFFu, m_new > m_run + kRescaleLog2)) {
-          // O must hold PV(g - 1) before it is rescaled
-          if (!wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) ok = false;
-          if (!__all_sync(0xFFFFFFFFu, ok)) {
+          // O must hold PV(g - 1) before it is rescaled (both warps of the
+          // quadrant take this branch: they hold the same row maxima)
+          const bool v_ok = __all_sync(0xFFFFFFFFu, wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1));
+          if (bar_red_or(1 + qd, 64, !v_ok)) {
             ok = false;
             break;
           }
@@ -485,19 +475,31 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
           }
         }
         // P = exp2(S * scale - m) as bf16: keys [c0, c0+64) -> columns [c0/2, c0/2+32)
+        // (in two 16-column halves: the first half's store runs while the
+        // second half is computed)
         float lsum = 0.f;
-        uint32_t pk[32];
+        {
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
-          float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
-          float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
-          float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
-          lsum += (p0 + p1) + (p2 + p3);
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-          pk[16 + (c >> 1)] = pack_bf16x2(p2, p3);
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2_approx(fmaf(a[c], p.scale_log2, -m_run));
+            const float p1 = ex2_approx(fmaf(a[c + 1], p.scale_log2, -m_run));
+            lsum += p0 + p1;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16u(s_col + hf * 32, pk);
         }
-        tmem_st32u(s_col + hf * 32, pk);
+        {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
+            const float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
+            lsum += p2 + p3;
+            pk[c >> 1] = pack_bf16x2(p2, p3);
+          }
+          tmem_st16u(s_col + hf * 32 + 16, pk);
+        }
         l_run += lsum;
         tmem_wait_st();
         tc_fence_before();
@@ -507,8 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
       }
       if (!ok) break;
       // hand the partial row sum to the epilogue once it is done with item t - 2
-      if (t >= 2 && !wait(&o_free[t & 1], ((t - 2) >> 1) & 1)) ok = false;
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
+      const bool f_ok = __all_sync(0xFFFFFFFFu, t < 2 || wait(&o_free[t & 1], ((t - 2) >> 1) & 1));
+      if (bar_red_or(1 + qd, 64, !f_ok)) {
         ok = false;
         break;
       }

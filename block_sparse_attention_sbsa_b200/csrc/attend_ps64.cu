@@ -31,7 +31,9 @@
 //              S(2), PV(1), ...
 //   warps 2-9  softmax: two warps per TMEM lane quadrant, 32 key columns
 //              each (the columns of their rows' half); the row maximum is
-//              exchanged through shared memory with the partner warp; the
+//              exchanged through shared memory with the partner warp at a
+//              named barrier of the two (which also tells both whether either
+//              has failed a bounded wait, so they leave together); the
 //              running maximum moves (and O is rescaled in TMEM) only when
 //              it grows by more than 2^8.
 //   warps 10-13 epilogue: O / l of the tile's 128 rows -> global memory.
@@ -67,8 +69,8 @@ struct PS64 {
   static constexpr int OFF_MX = OFF_L + 4 * BM * 4;          // row max [block%2][half][BM]
   static constexpr int OFF_BAR = OFF_MX + 4 * BM * 4;
   // q_full[2] q_free[2] kv_full[S] s_full[2] p_full[2] pv_done[2]
-  // o_full[2] o_free[2] l_full[2] mx_ready[2][4] drain
-  static constexpr int NBARS = 2 + 2 + kStages + 2 + 2 + 2 + 2 + 2 + 2 + 8 + 1;
+  // o_full[2] o_free[2] l_full[2] drain
+  static constexpr int NBARS = 2 + 2 + kStages + 2 + 2 + 2 + 2 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_S = 0;       // S[0], S[1]: 2 x BN columns
@@ -195,8 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
   uint64_t* o_full = pv_done + 2;
   uint64_t* o_free = o_full + 2;
   uint64_t* l_full = o_free + 2;
-  uint64_t* mx_ready = l_full + 2;  // [block % 2][quadrant]
-  uint64_t* drain = mx_ready + 8;
+  uint64_t* drain = l_full + 2;
   float* l_buf = reinterpret_cast<float*>(smem + C::OFF_L);
   float* mx_buf = reinterpret_cast<float*>(smem + C::OFF_MX);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -217,7 +218,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
       mbar_init(&o_full[b], 1);
       mbar_init(&o_free[b], 128);
       mbar_init(&l_full[b], 256);
-      for (int q = 0; q < 4; ++q) mbar_init(&mx_ready[b * 4 + q], 64);
     }
     for (int s = 0; s < kStages; ++s) mbar_init(&kv_full[s], 1);
     mbar_init(drain, 1);
@@ -376,6 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
     for (; ok && load_item(p, t, it, lane); ++t) {
       const int qb = t & 1;
       bool good = true;
+      // The warp reads the item's lists together (load_item); lane 0 alone
+      // waits and issues for the item's steps, and the outcome reaches the
+      // warp once per item.
       if (lane == 0) {
         good = wait(&q_full[qb], (t >> 1) & 1);
         if (good) {
@@ -386,15 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
             umma_commit(&o_full[qb]);
           }
         }
-      }
-      if (!warp_ok(good)) {
-        ok = false;
-        break;
-      }
-      if (it.steps == 0) continue;
-      for (int b = 0; b < it.steps; ++b) {
-        const bool last = (b == it.steps - 1);
-        if (lane == 0) {
+        for (int b = 0; good && b < it.steps; ++b) {
+          const bool last = (b == it.steps - 1);
           const int kpos = 2 * g;
           const int st = kpos % kStages;
           good = wait(&kv_full[st], (kpos / kStages) & 1);
@@ -416,14 +412,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
             if (last) umma_commit(&q_free[qb]);
             if (have_prev) good = issue_pv(prev);
           }
+          prev = Pending{g, t, b, last ? 1 : 0};
+          have_prev = true;
+          ++g;
         }
-        if (!warp_ok(good)) {
-          ok = false;
-          break;
-        }
-        prev = Pending{g, t, b, last ? 1 : 0};
-        have_prev = true;
-        ++g;
+      }
+      if (!warp_ok(good)) {
+        ok = false;
+        break;
       }
     }
     if (lane == 0) {
@@ -459,11 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
         // idle, the causal triangle on its diagonal block
         const int lim = jh < 0 ? -1 : (jh == 2 * it.m + half ? rl - hf * 32 : 31);
         const uint32_t s_col = tmem + lane_base + C::TM_S + (g & 1) * BN;
-        if (!wait(&s_full[g & 1], (g >> 1) & 1)) ok = false;
-        if (!__all_sync(0xFFFFFFFFu, ok)) {
-          ok = false;
-          break;
-        }
+        const bool s_ok = __all_sync(0xFFFFFFFFu, wait(&s_full[g & 1], (g >> 1) & 1));
         tc_fence_after();
         float a[32];
         tmem_ld32(s_col + c0, a);
@@ -483,9 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
         // finished reading S, so P may then overwrite the first S columns
         float* mxb = mx_buf + (g & 1) * 2 * BM;
         mxb[hf * BM + row] = mx;
-        mbar_arrive(&mx_ready[(g & 1) * 4 + qd]);
-        if (!wait(&mx_ready[(g & 1) * 4 + qd], (g >> 1) & 1)) ok = false;
-        if (!__all_sync(0xFFFFFFFFu, ok)) {
+        // the two warps of the quadrant meet once per step; the barrier also
+        // tells both whether either missed its S, so they leave together
+        if (bar_red_or(1 + qd, 64, !s_ok)) {
           ok = false;
           break;
         }
@@ -495,9 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
           if (b == 0) {
             m_run = m_new;
           } else if (__any_sync(0xFFFFFFFFu, m_new > m_run + kRescaleLog2)) {
-            // O must hold PV(g - 1) before it is rescaled
-            if (!wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) ok = false;
-            if (!__all_sync(0xFFFFFFFFu, ok)) {
+            // O must hold PV(g - 1) before it is rescaled (both warps of the
+            // quadrant take this branch: they hold the same row maxima)
+            const bool v_ok =
+                __all_sync(0xFFFFFFFFu, wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1));
+            if (bar_red_or(1 + qd, 64, !v_ok)) {
               ok = false;
               break;
             }
@@ -548,8 +542,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps64_kernel(const __grid_c
       }
       if (!ok) break;
       // hand the partial row sum to the epilogue once it is done with item t - 2
-      if (t >= 2 && !wait(&o_free[t & 1], ((t - 2) >> 1) & 1)) ok = false;
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
+      const bool f_ok = __all_sync(0xFFFFFFFFu, t < 2 || wait(&o_free[t & 1], ((t - 2) >> 1) & 1));
+      if (bar_red_or(1 + qd, 64, !f_ok)) {
         ok = false;
         break;
       }
