@@ -45,9 +45,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # kernel source it was taken on: once that source changes the figure no longer
 # describes the kernel and the line reports null.
 NCU_ATTEND_TRAFFIC = {
-    # profiles/attend_ps_kernel_dram_rbs.md: 2.36 GB read + 1.05 GB written
-    "rbs128k": {"bytes": 3.41e9, "source": "block_sparse_attention_sbsa_b200/csrc/attend_persist.cu",
-                "sha": "6bb6ffa558abafcc"},
+    # profiles/attend_ps_kernel_dram_rbs.md: 2.35 GB read + 1.05 GB written
+    "rbs128k": {"bytes": 3.40e9, "source": "block_sparse_attention_sbsa_b200/csrc/attend_persist.cu",
+                "sha": "2772f1140986d557"},
 }
 
 

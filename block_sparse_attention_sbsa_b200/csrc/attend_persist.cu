@@ -37,6 +37,10 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+#include <cstring>
+
+#include "exp2_fma.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 #include "tma_map.h"
@@ -152,7 +156,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int D>
+// kFmaExp: one exponential in four on the FMA pipe (exp2_fma), the rest on
+// the MUFU; an option, not the default (measured slower on the B200).
+template <int D, bool kFmaExp>
 __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_constant__ PSParams p) {
   using C = PS<D>;
   constexpr int BM = C::BM, BN = C::BN;
@@ -494,7 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const float p2 = ex2_approx(fmaf(bb[c], p.scale_log2, -m_run));
-            const float p3 = ex2_approx(fmaf(bb[c + 1], p.scale_log2, -m_run));
+            const float x3 = fmaf(bb[c + 1], p.scale_log2, -m_run);
+            const float p3 = kFmaExp ? exp2_fma(x3) : ex2_approx(x3);
             lsum += p2 + p3;
             pk[c >> 1] = pack_bf16x2(p2, p3);
           }
@@ -576,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ps_kernel(const __grid_con
 }
 
 template <int D>
-int launch_d(const AttendArgs& a, cudaStream_t stream) {
+int launch_d(const AttendArgs& a, cudaStream_t stream, bool fma_exp) {
   using C = PS<D>;
   PSParams p{};
   const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -596,7 +603,7 @@ int launch_d(const AttendArgs& a, cudaStream_t stream) {
   p.total = a.hq * p.nb;
   p.scale_log2 = a.sm_scale * 1.4426950408889634f;
   p.status = a.status;
-  auto kern = attend_ps_kernel<D>;
+  auto kern = fma_exp ? attend_ps_kernel<D, true> : attend_ps_kernel<D, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return SBSA_ERR_CUDA;
@@ -607,13 +614,32 @@ int launch_d(const AttendArgs& a, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? SBSA_OK : SBSA_ERR_CUDA;
 }
 
+__global__ void exp2_fma_kernel(const float* x, float* y, long long n) {
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x)
+    y[e] = exp2_fma(x[e]);
+}
+
 }  // namespace
 
 int launch_attend_persistent(const AttendArgs& a, cudaStream_t stream) {
+  // SBSA_ATTEND_EXP2=fma takes one exponential in four on the FMA pipe
+  static const bool fma_exp = [] {
+    const char* e = std::getenv("SBSA_ATTEND_EXP2");
+    return e != nullptr && std::strcmp(e, "fma") == 0;
+  }();
   if (a.dtype != SBSA_BF16 || a.block != 128) return SBSA_ERR_UNSUPPORTED;
-  if (a.d == 128) return launch_d<128>(a, stream);
-  if (a.d == 64) return launch_d<64>(a, stream);
+  if (a.d == 128) return launch_d<128>(a, stream, fma_exp);
+  if (a.d == 64) return launch_d<64>(a, stream, fma_exp);
   return SBSA_ERR_UNSUPPORTED;
+}
+
+cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const long long blocks = (n + 255) / 256;
+  const int grid = blocks < 4096 ? (int)blocks : 4096;
+  exp2_fma_kernel<<<grid, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
 }
 
 }  // namespace sbsa

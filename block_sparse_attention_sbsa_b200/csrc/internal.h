@@ -135,6 +135,9 @@ int launch_attend_single(const AttendArgs& a, cudaStream_t stream);
 
 // The persistent pipelined kernel (bf16, B = 128, d in {64, 128}).
 int launch_attend_persistent(const AttendArgs& a, cudaStream_t stream);
+// exp2_fma (the FMA-pipe exponential the persistent kernel can use for a
+// part of its softmax) applied to n floats in device memory.
+cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t stream);
 
 // The persistent pipelined kernel on tiles of two 64-token query blocks
 // (bf16, B = 64, d in {64, 128}).

@@ -640,6 +640,13 @@ int sbsa_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
                                      static_cast<cudaStream_t>(stream)));
 }
 
+int sbsa_exp2_fma_eval(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0) return SBSA_ERR_INVALID_ARG;
+  if (n == 0) return SBSA_OK;
+  if (!x || !y) return SBSA_ERR_INVALID_ARG;
+  return cuda_code(launch_exp2_fma(x, y, (long long)n, static_cast<cudaStream_t>(stream)));
+}
+
 int sbsa_get_status(void* stream, int* device_status) {
   if (!device_status) return SBSA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)

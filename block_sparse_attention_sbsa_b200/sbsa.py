@@ -33,7 +33,7 @@ SYMBOLS = ["sbsa_pool_blocks", "sbsa_pool_minmax", "sbsa_select", "sbsa_select_w
            "sbsa_select_scores", "sbsa_select_gate_partial", "sbsa_select_gate_finish",
            "sbsa_attend", "sbsa_prefill", "sbsa_prefill_host", "sbsa_prefill_host_workspace_bytes",
            "sbsa_prefill_workspace_bytes", "sbsa_get_status", "sbsa_status_string",
-           "sbsa_version", "sbsa_debug_wait_timeout"]
+           "sbsa_version", "sbsa_debug_wait_timeout", "sbsa_exp2_fma_eval"]
 
 
 class SbsaError(RuntimeError):
@@ -119,6 +119,7 @@ def _load() -> ctypes.CDLL:
     lib.sbsa_status_string.restype = ctypes.c_char_p
     lib.sbsa_version.argtypes = []
     lib.sbsa_debug_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.sbsa_exp2_fma_eval.argtypes = [f32p, f32p, ctypes.c_int64, vp]
     for name in ["sbsa_pool_blocks", "sbsa_select", "sbsa_attend", "sbsa_prefill",
                  "sbsa_get_status", "sbsa_version", "sbsa_debug_wait_timeout"]:
         getattr(lib, name).restype = ctypes.c_int
@@ -420,6 +421,18 @@ def debug_wait_timeout(timeout_ns: int, stream=None):
     """Launch the bounded-wait probe (see include/sbsa.h)."""
     _check(lib.sbsa_debug_wait_timeout(int(timeout_ns), _stream(stream)),
            "sbsa_debug_wait_timeout")
+
+
+def exp2_fma_eval(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """exp2 on the FMA pipe (the attention softmax's option) of each element
+    of a float32 CUDA tensor (see include/sbsa.h)."""
+    if x.dtype != torch.float32 or not x.is_cuda:
+        raise ValueError("x must be a float32 CUDA tensor")
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    _check(lib.sbsa_exp2_fma_eval(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "sbsa_exp2_fma_eval")
+    return y
 
 
 def get_status(stream=None) -> int:

@@ -365,6 +365,20 @@ int sbsa_version(void);
 int sbsa_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
 /*
+ * sbsa_exp2_fma_eval -- test hook for the exponential that the persistent
+ * 128-token attention kernel can take on the FMA pipe for one score in four
+ * (the option SBSA_ATTEND_EXP2=fma in the environment; the default keeps
+ * every exponential on the MUFU).  [RBS] method paragraph: the prefill's
+ * softmax.  Writes y[e] = exp2_fma(x[e]) for e < n: Cody-Waite reduction
+ * x = n + f, f in [-1/2, 1/2], and a degree-3 minimax polynomial for 2^f,
+ * relative error below 7.5e-5 for x in [-125, 8], exactly 0 below -125.
+ *   x, y  device fp32 [n]; may not overlap unless equal.
+ *   n     elements; 0 enqueues nothing.
+ * Returns SBSA_ERR_INVALID_ARG for n < 0 or a NULL pointer with n > 0.
+ */
+int sbsa_exp2_fma_eval(const float* x, float* y, int64_t n, void* stream);
+
+/*
  * sbsa_prefill_noalloc -- sbsa_prefill for callers that cannot allocate
  * device memory.  The pages have no counterpart: this is a deployment
  * convenience of this library.
