@@ -27,8 +27,9 @@
 // TMEM with P aliased into it; Q and O are double-buffered per item.  14 warps:
 //   warp 0     TMA producer (Q of item t into Q[t % 2]; the two K blocks and
 //              the two V blocks of step g into ring positions 2g, 2g + 1).
-//   warp 1     TMEM owner and single-thread MMA issuer: S(0), S(1), PV(0),
-//              S(2), PV(1), ...
+//   warp 1     TMEM owner and single-thread MMA issuer (the warp reads each
+//              item's lists together, then lane 0 alone waits and issues for
+//              the item's steps): S(0), S(1), PV(0), S(2), PV(1), ...
 //   warps 2-9  softmax: two warps per TMEM lane quadrant, 32 key columns
 //              each (the columns of their rows' half); the row maximum is
 //              exchanged through shared memory with the partner warp at a

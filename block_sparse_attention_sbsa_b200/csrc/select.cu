@@ -17,9 +17,12 @@
 // Componibilidad: Quest-style per-coordinate upper bounds), from
 // sum_d max(q_d min_d, q_d max_d) over the block's coordinate box.
 //
-// Layout of one CTA: R (up to 16) consecutive query blocks of one selection
-// head.  Phase 1 puts their scores against every earlier key block into
-// shared memory: copied from a precomputed table (the tensor-core centroid
+// Layout of one CTA: R consecutive query blocks of one selection head (8
+// when the scores come from a table, up to 16 when they are computed here).
+// The rows' pooled queries, the kv head's radii and the table's score rows
+// are staged into shared memory by bulk copies on one barrier when aligned.
+// Phase 1 puts their scores against every earlier key block into shared
+// memory: copied from a precomputed table (the tensor-core centroid
 // scores, or the row-max tile scores), or computed here -- each thread
 // streams whole key-centroid rows from L2 in 16-byte pieces and dots them
 // with the R pooled queries held in shared memory (fp32 FMA; each centroid
