@@ -112,3 +112,24 @@ def test_attention_with_fma_exponentials_matches_oracle():
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
                        text=True, timeout=600)
     assert r.returncode == 0 and "fma ok" in r.stdout, r.stdout + r.stderr
+
+
+def test_eval_entry_rejects_bad_arguments_on_the_host():
+    """sbsa_exp2_fma_eval checks its arguments before any CUDA call."""
+    import ctypes
+    from block_sparse_attention_sbsa_b200 import sbsa
+    fake = ctypes.c_void_p(0x10000)
+    assert sbsa.lib.sbsa_exp2_fma_eval(fake, fake, -1, None) == sbsa.ERR_INVALID_ARG
+    assert sbsa.lib.sbsa_exp2_fma_eval(None, fake, 4, None) == sbsa.ERR_INVALID_ARG
+    assert sbsa.lib.sbsa_exp2_fma_eval(fake, None, 4, None) == sbsa.ERR_INVALID_ARG
+    # nothing to do: no launch, no pointer needed
+    assert sbsa.lib.sbsa_exp2_fma_eval(None, None, 0, None) == sbsa.OK
+
+
+def test_binding_rejects_non_float32_or_host_tensors():
+    import torch
+    from block_sparse_attention_sbsa_b200 import sbsa
+    with pytest.raises(ValueError):
+        sbsa.exp2_fma_eval(torch.zeros(4, dtype=torch.float32))  # host memory
+    with pytest.raises(ValueError):
+        sbsa.exp2_fma_eval(torch.zeros(4, dtype=torch.float64))
